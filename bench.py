@@ -1,0 +1,368 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused, chunked distillation KL loss (forward + backward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kernels|reference]
+
+One step = one kl_fwd_bwd call (top-K prep, logits + split-V statistics with the
+fused cache gather, row merge, dlogits, dH and dW contractions, loss mean) over
+one batch of the offline top-K workload: N=4096 tokens, d=3072, V=128256, bf16,
+teacher cache K=64 (int32 ids + fp32 logits + fp32 teacher log-sum-exp, partial
+mass kept), T=1.  Inputs are synthetic and seeded; W (0.79 GB) and the logit
+chunk (1.05 GB) are larger than the 126 MB L2, so no flush is needed between
+steps.  With --gpus N (under torchrun) every rank runs its own N=4096-token
+shard with no collective on the data path (weak scaling); the elapsed time is
+the max over ranks.
+
+Prints ONE JSON line on rank 0.  `--impl reference` times the fp64 CPU oracle
+instead, on the host cores, on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused KL fwd+bwd tokens/s at V=128256,d=3072; % bf16 TC peak; extra HBM GiB"
+WORKLOAD = ("offline top-K KD: N=4096 tokens, d=3072, V=128256, bf16 H~N(0,1), "
+            "W~N(0,0.02^2); cache K=64 int32 ids + fp32 logits + fp32 teacher lse "
+            "(partial mass) from a bf16 teacher head d_t=4096; T=1")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kernels", choices=["kernels", "reference"])
+    ap.add_argument("--N", type=int, default=4096)
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=0,
+                    help="tokens in the oracle sample (0 = sized to ~10 s)")
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import chunked_kl_loss_tma_b200 as ckl
+    from chunked_kl_loss_tma_b200 import _lib, ops
+    from chunked_kl_loss_tma_b200 import workloads as wl
+
+    ws, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    w = wl.offline_topk(device=dev, N=args.N, seed=1 + rank)
+    torch.cuda.empty_cache()  # drop the teacher-cache generator's temporaries
+    kw = dict(T=w.T, topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse,
+              chunk_tokens=args.chunk)
+    prob, keep = ops.make_problem(w.H, w.W, **kw)
+    ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
+    torch.cuda.synchronize()
+    base_mem = torch.cuda.memory_allocated(dev)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    dH = torch.empty_like(w.H)
+    dW = torch.empty(w.W.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+
+    def step():
+        _lib.check(_lib.kl_fwd_bwd(prob, workspace.data_ptr(), ws_bytes, 1.0, loss.data_ptr(),
+                                   None, dH.data_ptr(), dW.data_ptr(), 0, stream), "kl_fwd_bwd")
+
+    torch.cuda.reset_peak_memory_stats(dev)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    status = _lib.kl_status(workspace.data_ptr(), stream)
+    if status != 0:
+        raise RuntimeError(f"device status {_lib.STATUS.get(status)} after warm-up")
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = _lib.kl_launch_count()
+    _lib.kl_profile_begin()
+    barrier()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    barrier()
+    prof = _lib.kl_profile_end()
+    launches = _lib.kl_launch_count() - launches0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    peak_extra = torch.cuda.max_memory_allocated(dev) - base_mem
+    elapsed = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(elapsed, op=dist.ReduceOp.MAX)
+    ms = float(elapsed.item())
+
+    # ---- end to end through the public API: pinned host inputs in, loss out
+    e2e = None
+    if not args.no_e2e:
+        hH = w.H.cpu().pin_memory()
+        hidx = w.topk_idx.cpu().pin_memory()
+        hval = w.topk_logit.cpu().pin_memory()
+        hlse = w.teacher_lse.cpu().pin_memory()
+        hloss = torch.empty((), dtype=torch.float32).pin_memory()
+        dHin, didx, dval, dlse = (torch.empty_like(w.H), torch.empty_like(w.topk_idx),
+                                  torch.empty_like(w.topk_logit), torch.empty_like(w.teacher_lse))
+        prob2, keep2 = ops.make_problem(dHin, w.W, T=w.T, topk_idx=didx, topk_logit=dval,
+                                        teacher_lse=dlse, chunk_tokens=args.chunk)
+
+        def e2e_step():
+            dHin.copy_(hH, non_blocking=True)
+            didx.copy_(hidx, non_blocking=True)
+            dval.copy_(hval, non_blocking=True)
+            dlse.copy_(hlse, non_blocking=True)
+            _lib.check(_lib.kl_fwd_bwd(prob2, workspace.data_ptr(), ws_bytes, 1.0,
+                                       loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(), 0,
+                                       stream), "kl_fwd_bwd")
+            hloss.copy_(loss, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        barrier()
+        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        h2d = sum(t.numel() * t.element_size() for t in (hH, hidx, hval, hlse))
+        e2e = {"value": ws * args.N * args.steps / (float(ems.item()) / 1e3),
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = measured_peaks()
+    N, d, V = args.N, 3072, 128256
+    tok_s = ws * N * args.steps / (ms / 1e3)
+    dom = max(prof, key=lambda p: p["total_ms"]) if prof else None
+    roof = None
+    if dom is not None:
+        per_launch_flops = dom["flops"] / max(dom["launches"], 1)
+        avg_s = dom["total_ms"] / max(dom["launches"], 1) / 1e3
+        if per_launch_flops > 0:
+            achieved = per_launch_flops / avg_s / 1e12
+            peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+            roof = {"kernel": dom["name"], "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "traffic": None,
+                    "peak_source": f"{peak_src} sustained bf16 (kernel timed inside a long step)",
+                    "avg_launch_ms": round(avg_s * 1e3, 4),
+                    "flops_per_launch": per_launch_flops}
+        else:
+            achieved = dom["bytes"] / max(dom["launches"], 1) / avg_s / 1e9
+            roof = {"kernel": dom["name"], "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+    step_flops = 6.0 * N * d * V
+    step_tflops = step_flops * args.steps / (ms / 1e3) / 1e12
+    kernels = {p["name"]: {"launches": p["launches"], "ms": round(p["total_ms"], 3),
+                           "share": round(p["total_ms"] / sum(q["total_ms"] for q in prof), 4)}
+               for p in prof}
+    line = {
+        "metric": METRIC, "value": round(tok_s, 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init heads and teacher cache)",
+        "config": {"workload": WORKLOAD, "N_per_gpu": N, "d": d, "V": V, "K": 64, "T": 1.0,
+                   "chunk_tokens": args.chunk or min(4096, N),
+                   "l2": "inputs larger than L2 (W 0.79 GB, logit chunk 1.05 GB); no flush",
+                   "parallelism": f"weak-scaling token shards x{ws}, no data-path collective"},
+        "tensor_tflops_step": round(step_tflops, 1),
+        "tensor_frac_step": round(step_tflops / peaks.get("bf16_tflops_sustained", 1400.0), 4),
+        "tensor_frac_step_burst_peak": round(step_tflops / peaks.get("bf16_tflops", 1590.0), 4),
+        "tensor_frac_step_spec_2250": round(step_tflops / 2250.0, 4),
+        "extra_hbm_gib": round(ws_bytes / 2**30, 4),
+        "extra_hbm_gib_measured_peak": round(peak_extra / 2**30, 4),
+        "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clk,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
+    print(json.dumps(line), flush=True)
+
+
+def _oracle_sample(w, n_tokens):
+    """The oracle on the first n_tokens rows of the workload as a problem of its
+    own (loss, dH and dW over those rows)."""
+    import oracle
+
+    sl = slice(0, n_tokens)
+    return oracle.kl_loss(w.H[sl], w.W, T=w.T, mode="topk", topk_idx=w.topk_idx[sl],
+                          topk_logit=w.topk_logit[sl], teacher_lse=w.teacher_lse[sl])
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(w, n_tokens=0):
+    """fp64 oracle throughput on the host cores over a bounded token sample."""
+    import numpy as np
+
+    Wd = w.W.cpu()
+    sample = w.to("cpu")
+    sample.W = Wd
+    t0 = time.time()
+    _oracle_sample(sample, 8)
+    t_probe = time.time() - t0
+    if n_tokens <= 0:
+        n_tokens = int(np.clip(8 * 10.0 / max(t_probe, 1e-3), 8, 512))
+    t0 = time.time()
+    _oracle_sample(sample, n_tokens)
+    dt = time.time() - t0
+    return {"value": round(n_tokens / dt, 3), "unit": "tokens/s", "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"first {n_tokens} tokens of the workload as a problem of their own "
+                      f"(fp64 loss, dH and dW; {dt:.1f} s)"}
+
+
+def reference_arm(args):
+    ws, rank, local = dist_setup(args)
+    if rank != 0:
+        return
+    import torch
+
+    from chunked_kl_loss_tma_b200 import workloads as wl
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = wl.offline_topk(device=dev, N=args.N, seed=1).to("cpu")
+    per_step = args.cpu_sample or 16
+    for _ in range(max(args.warmup, 3)):
+        _oracle_sample(w, 2)
+    t0 = time.time()
+    for _ in range(args.steps):
+        _oracle_sample(w, per_step)
+    dt = time.time() - t0
+    v = per_step * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "N_per_gpu": args.N,
+                   "sample_per_step": f"{per_step} tokens (fp64 oracle on host cores)"},
+        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": _cores(),
+                         "kind": "oracle",
+                         "sample": f"{per_step} tokens per step of the same workload"},
+        "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,830 @@
+// kl_api.cu -- C ABI of the fused, chunked distillation KL loss (sm_100a).
+//
+// Host side: argument validation, workspace planning, TMA tensor-map encoding
+// and the per-chunk launch sequence ("Efficient Knowledge Distillation for
+// LLMs: Offline Top-K Logits and a Fused Chunked KL Loss", §3 "Fused chunked
+// KL": the output projection is fused into the loss, each logit chunk is
+// transient, and backward recomputes one projection per chunk).
+//
+// Per chunk of C token rows (fwd_bwd, top-K):
+//   prep_topk      cache -> sorted ids + teacher probabilities q, m, sum q log q
+//   gemm STATS     S~ = H_c W^T / T  (tcgen05), split-V row statistics + gather
+//   row_reduce     lse_s, row loss
+//   dlogits_topk   S~ -> dS in place
+//   gemm STORE     dH_c = dS W
+//   gemm ACCUM     dW (+)= dS^T H_c
+// then finalize_loss (masked mean).  No host synchronisation anywhere.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/chunked_kl.h"
+#include "kl_gemm.cuh"
+#include "kl_rowops.cuh"
+
+using namespace ckl;
+
+namespace {
+
+// ------------------------------------------------------------------ device
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+  int checked = 0;
+  int ok = 0;
+  int sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return KL_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.checked = 1;
+  }
+  *out = d;
+  return d.ok ? KL_OK : KL_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major matrix [rows][inner] with the given row stride,
+// 128-byte swizzle, zero fill outside the extents.
+bool make_map(CUtensorMap* m, const void* base, int dtype, uint64_t inner, uint64_t rows,
+              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(m, dtype == KL_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+         2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ profiling
+std::atomic<uint64_t> g_launches{0};
+
+struct ProfKind {
+  std::string name;
+  uint64_t launches = 0;
+  double flops = 0, bytes = 0;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfKind> g_prof;
+std::vector<cudaEvent_t> g_ev_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct LaunchScope {
+  cudaStream_t st;
+  ProfKind* kind = nullptr;
+  cudaEvent_t e0 = nullptr;
+  LaunchScope(const char* name, cudaStream_t s, double flops, double bytes) : st(s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_on) return;
+    for (auto& k : g_prof)
+      if (k.name == name) kind = &k;
+    if (kind == nullptr) {
+      g_prof.push_back(ProfKind());
+      kind = &g_prof.back();
+      kind->name = name;
+    }
+    kind->launches++;
+    kind->flops += flops;
+    kind->bytes += bytes;
+    e0 = pool_event();
+    cudaEventRecord(e0, st);
+  }
+  ~LaunchScope() {
+    if (kind == nullptr) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t e1 = pool_event();
+    cudaEventRecord(e1, st);
+    kind->ev.emplace_back(e0, e1);
+  }
+};
+
+long long spin_limit() {
+  static long long lim = [] {
+    const char* s = getenv("KL_SPIN_LIMIT");
+    long long v = s ? atoll(s) : 0;
+    return v > 0 ? v : 4000000000LL;  // ~2 s at the B200 boost clock
+  }();
+  return lim;
+}
+
+#define KL_TRY(x)                 \
+  do {                            \
+    const int _e = (x);           \
+    if (_e != KL_OK) return _e;   \
+  } while (0)
+
+// ------------------------------------------------------------------ planning
+constexpr int64_t kDefaultChunk = 4096;
+constexpr int kMaxK = 1024;
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int eb = 2;          // element bytes
+  int64_t C = 0;       // chunk rows
+  int64_t Vp = 0;      // padded logit-buffer row length (multiple of 8)
+  int tiles_v = 0;     // 256-column tiles over V
+  bool hidden = false;
+  // workspace offsets (bytes)
+  size_t off_sbuf = 0, off_tbuf = 0, off_ps = 0, off_pt = 0, off_sidx = 0, off_sq = 0,
+         off_rinfo = 0, off_lse_s = 0, off_lse_t = 0, off_rl = 0, total = 0;
+  // fp32 (tf32) path only: tf32-rounded operand copies (heads W, Wt; the
+  // current chunk of H or Ht) and K-major copies W^T [d][Vp], dS^T [V][Cp],
+  // H_c^T [d][Cp] for the gradient contractions.
+  int64_t Cp = 0;
+  size_t off_wr = 0, off_wtr = 0, off_xr = 0, off_wT = 0, off_sT = 0, off_hT = 0;
+};
+
+// Sizes, dtypes and scalar arguments (no pointers).
+int validate_shape(const kl_problem* p) {
+  if (p == nullptr) return KL_ERR_NULL;
+  if (p->dtype != KL_DTYPE_BF16 && p->dtype != KL_DTYPE_F32) return KL_ERR_DTYPE;
+  if (p->teacher != KL_TEACHER_TOPK && p->teacher != KL_TEACHER_HIDDEN) return KL_ERR_DTYPE;
+  if (p->N < 0 || p->d < 1 || p->V < 1 || p->N > (int64_t(1) << 31) - 1 ||
+      p->V > (int64_t(1) << 31) - 512 || p->d > (int64_t(1) << 20))
+    return KL_ERR_SHAPE;
+  if (!(p->T > 0.f) || !(p->T < INFINITY) || p->chunk_tokens < 0 || !(p->normalizer >= 0.f))
+    return KL_ERR_ARG;
+  if (p->d % 8 != 0) return KL_ERR_ALIGN;
+  if (p->teacher == KL_TEACHER_TOPK) {
+    if (p->K < 1 || p->K > kMaxK) return KL_ERR_SHAPE;
+  } else {
+    if (p->d_t < 1 || p->d_t > (int64_t(1) << 20)) return KL_ERR_SHAPE;
+    if (p->d_t % 8 != 0) return KL_ERR_ALIGN;
+  }
+  return KL_OK;
+}
+
+int validate(const kl_problem* p) {
+  KL_TRY(validate_shape(p));
+  if (p->N > 0) {
+    if (p->H == nullptr || p->W == nullptr) return KL_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(p->H) | reinterpret_cast<uintptr_t>(p->W)) & 15)
+      return KL_ERR_ALIGN;
+    if (p->teacher == KL_TEACHER_TOPK) {
+      if (p->topk_idx == nullptr || p->topk_logit == nullptr) return KL_ERR_NULL;
+    } else {
+      if (p->Ht == nullptr || p->Wt == nullptr) return KL_ERR_NULL;
+      if ((reinterpret_cast<uintptr_t>(p->Ht) | reinterpret_cast<uintptr_t>(p->Wt)) & 15)
+        return KL_ERR_ALIGN;
+    }
+  }
+  return KL_OK;
+}
+
+Plan make_plan(const kl_problem* p, int entry) {
+  Plan pl;
+  pl.eb = p->dtype == KL_DTYPE_BF16 ? 2 : 4;
+  pl.hidden = p->teacher == KL_TEACHER_HIDDEN;
+  const int64_t chunk = p->chunk_tokens > 0 ? p->chunk_tokens : kDefaultChunk;
+  pl.C = p->N < chunk ? p->N : chunk;
+  if (pl.C < 1) pl.C = 1;
+  pl.Vp = cdiv(p->V, 8) * 8;
+  pl.tiles_v = static_cast<int>(cdiv(p->V, kBN));
+  const bool need_sbuf = entry != KL_ENTRY_FWD || pl.hidden;
+  const bool need_stats = entry != KL_ENTRY_BWD;
+  size_t off = 256;  // Scalars
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  const size_t buf = static_cast<size_t>(pl.C) * pl.Vp * pl.eb;
+  if (need_sbuf) pl.off_sbuf = take(buf);
+  if (need_sbuf && pl.hidden) pl.off_tbuf = take(buf);
+  if (need_stats) pl.off_ps = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
+  if (need_stats && pl.hidden)
+    pl.off_pt = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
+  if (!pl.hidden) {
+    pl.off_sidx = take(static_cast<size_t>(pl.C) * p->K * 4);
+    pl.off_sq = take(static_cast<size_t>(pl.C) * p->K * 4);
+    pl.off_rinfo = take(static_cast<size_t>(pl.C) * sizeof(float2));
+  }
+  const size_t nrow = static_cast<size_t>(p->N > 0 ? p->N : 1) * 4;
+  if (entry == KL_ENTRY_FWD_BWD) {
+    pl.off_lse_s = take(nrow);
+    if (pl.hidden) pl.off_lse_t = take(nrow);
+  }
+  if (entry != KL_ENTRY_BWD) pl.off_rl = take(nrow);
+  if (pl.eb == 4) {
+    const int64_t dmax = (pl.hidden && p->d_t > p->d) ? p->d_t : p->d;
+    pl.off_wr = take(static_cast<size_t>(p->V) * p->d * 4);
+    if (pl.hidden) pl.off_wtr = take(static_cast<size_t>(p->V) * p->d_t * 4);
+    pl.off_xr = take(static_cast<size_t>(pl.C) * dmax * 4);
+  }
+  if (pl.eb == 4 && entry != KL_ENTRY_FWD) {
+    pl.Cp = cdiv(pl.C, 4) * 4;
+    pl.off_wT = take(static_cast<size_t>(p->d) * pl.Vp * 4);
+    pl.off_sT = take(static_cast<size_t>(p->V) * pl.Cp * 4);
+    pl.off_hT = take(static_cast<size_t>(p->d) * pl.Cp * 4);
+  }
+  pl.total = off;
+  return pl;
+}
+
+// ------------------------------------------------------------------ launches
+template <typename Elem, int A_MN, int B_MN, int EPI>
+int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
+                const CUtensorMap& mb, GemmParams gp, double flops) {
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
+        cudaSuccess)
+      return KL_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int tiles = gp.tiles_m * gp.tiles_n;
+  const int grid = tiles < sms ? tiles : sms;
+  {
+    LaunchScope ls(name, st, flops, 0);
+    kern<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(ma, mb, gp);
+  }
+  return cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA;
+}
+
+#define KL_LAUNCHED() (cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA)
+
+struct Ctx {
+  const kl_problem* p;
+  Plan pl;
+  uint8_t* ws;
+  Scalars* sc;
+  cudaStream_t st;
+  int sms;
+  float invT;
+};
+
+int launch_round(Ctx& c, const float* src, int64_t ld_src, float* dst, int64_t ld_dst,
+                 int64_t rows, int64_t cols) {
+  LaunchScope ls("round_tf32", c.st, 0, 8.0 * rows * cols);
+  round_tf32_kernel<<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(src, ld_src, dst, ld_dst,
+                                                                       rows, cols);
+  return cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA;
+}
+
+// Heads as the logits contraction reads them (tf32-rounded copies for fp32).
+const void* head_W(Ctx& c) {
+  return c.pl.eb == 4 ? static_cast<const void*>(c.ws + c.pl.off_wr) : c.p->W;
+}
+const void* head_Wt(Ctx& c) {
+  return c.pl.eb == 4 ? static_cast<const void*>(c.ws + c.pl.off_wtr) : c.p->Wt;
+}
+int prepare_heads(Ctx& c) {
+  if (c.pl.eb != 4) return KL_OK;
+  const kl_problem* p = c.p;
+  KL_TRY(launch_round(c, static_cast<const float*>(p->W), p->d,
+                      reinterpret_cast<float*>(c.ws + c.pl.off_wr), p->d, p->V, p->d));
+  if (c.pl.hidden)
+    KL_TRY(launch_round(c, static_cast<const float*>(p->Wt), p->d_t,
+                        reinterpret_cast<float*>(c.ws + c.pl.off_wtr), p->d_t, p->V, p->d_t));
+  return KL_OK;
+}
+
+template <typename Elem>
+int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, int64_t Cn,
+                void* out, float4* partials, const int* sidx, const float* sq, int ktop,
+                const char* name) {
+  const kl_problem* p = c.p;
+  constexpr int kBKe = kRowBytes / sizeof(Elem);
+  CUtensorMap ma, mb;
+  const uint8_t* xc = static_cast<const uint8_t*>(X) + c0 * dx * sizeof(Elem);
+  if (sizeof(Elem) == 4) {  // tf32: round the chunk of hidden states first
+    float* xr = reinterpret_cast<float*>(c.ws + c.pl.off_xr);
+    KL_TRY(launch_round(c, reinterpret_cast<const float*>(xc), dx, xr, dx, Cn, dx));
+    xc = reinterpret_cast<const uint8_t*>(xr);
+  }
+  if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
+      !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN))
+    return KL_ERR_CUDA;
+  GemmParams gp{};
+  gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+  gp.tiles_n = c.pl.tiles_v;
+  gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
+  gp.m_fastest = 1;
+  gp.out = out;
+  gp.ld_out = c.pl.Vp;
+  gp.rows_valid = static_cast<int>(Cn);
+  gp.cols_valid = static_cast<int>(p->V);
+  gp.cols_store = static_cast<int>(c.pl.Vp);
+  gp.scale = c.invT;
+  gp.partials = partials;
+  gp.sidx = sidx;
+  gp.sq = sq;
+  gp.ktop = ktop;
+  gp.status = &c.sc->status;
+  gp.spin_limit = spin_limit();
+  return launch_gemm<Elem, 0, 0, EPI_STATS>(name, c.st, c.sms, ma, mb, gp,
+                                            2.0 * Cn * p->V * dx);
+}
+
+int launch_transpose(Ctx& c, const float* src, int64_t ld_src, float* dst, int64_t ld_dst,
+                     int64_t rows, int64_t cols) {
+  LaunchScope ls("transpose_f32", c.st, 0, 8.0 * rows * cols);
+  dim3 grid(static_cast<unsigned>(cdiv(cols, 32)), static_cast<unsigned>(cdiv(rows, 32)));
+  transpose_f32_kernel<<<grid, dim3(32, 8), 0, c.st>>>(src, ld_src, dst, ld_dst,
+                                                       static_cast<int>(rows),
+                                                       static_cast<int>(cols));
+  return cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA;
+}
+
+// fp32 inputs: both gradient contractions with K-major tf32 operands only.
+int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta) {
+  const kl_problem* p = c.p;
+  const int64_t d = p->d, V = p->V, Cp = c.pl.Cp;
+  float* sT = reinterpret_cast<float*>(c.ws + c.pl.off_sT);
+  float* hT = reinterpret_cast<float*>(c.ws + c.pl.off_hT);
+  const float* wT = reinterpret_cast<const float*>(c.ws + c.pl.off_wT);
+  const float* hc = static_cast<const float*>(p->H) + c0 * d;
+  KL_TRY(launch_transpose(c, dS, c.pl.Vp, sT, Cp, Cn, V));
+  KL_TRY(launch_transpose(c, hc, d, hT, Cp, Cn, d));
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dS, p->dtype, V, Cn, c.pl.Vp * 4, 32, kBM) ||
+        !make_map(&mb, wT, p->dtype, V, d, c.pl.Vp * 4, 32, kBN))
+      return KL_ERR_CUDA;
+    GemmParams gp{};
+    gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+    gp.tiles_n = static_cast<int>(cdiv(d, kBN));
+    gp.num_kb = static_cast<int>(cdiv(V, 32));
+    gp.m_fastest = 1;
+    gp.out = static_cast<float*>(dH) + c0 * d;
+    gp.ld_out = d;
+    gp.rows_valid = static_cast<int>(Cn);
+    gp.cols_valid = static_cast<int>(d);
+    gp.status = &c.sc->status;
+    gp.spin_limit = spin_limit();
+    KL_TRY((launch_gemm<float, 0, 0, EPI_STORE>("gemm_dH", c.st, c.sms, ma, mb, gp,
+                                                2.0 * Cn * V * d)));
+  }
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, sT, p->dtype, Cn, V, Cp * 4, 32, kBM) ||
+        !make_map(&mb, hT, p->dtype, Cn, d, Cp * 4, 32, kBN))
+      return KL_ERR_CUDA;
+    GemmParams gp{};
+    gp.tiles_m = static_cast<int>(cdiv(V, kBM));
+    gp.tiles_n = static_cast<int>(cdiv(d, kBN));
+    gp.num_kb = static_cast<int>(cdiv(Cn, 32));
+    gp.m_fastest = 0;
+    gp.out = dW;
+    gp.ld_out = d;
+    gp.rows_valid = static_cast<int>(V);
+    gp.cols_valid = static_cast<int>(d);
+    gp.beta = beta;
+    gp.status = &c.sc->status;
+    gp.spin_limit = spin_limit();
+    KL_TRY((launch_gemm<float, 0, 0, EPI_ACCUM>("gemm_dW", c.st, c.sms, ma, mb, gp,
+                                                2.0 * Cn * V * d)));
+  }
+  return KL_OK;
+}
+
+template <typename Elem>
+int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta) {
+  if (sizeof(Elem) == 4)
+    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
+  const kl_problem* p = c.p;
+  constexpr int kBKe = kRowBytes / sizeof(Elem);
+  constexpr int kMNe = kRowBytes / sizeof(Elem);
+  const int64_t d = p->d;
+  const uint64_t ldS = c.pl.Vp * sizeof(Elem);
+  // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kBKe, kBM) ||
+        !make_map(&mb, p->W, p->dtype, d, p->V, d * sizeof(Elem), kMNe, kBKe))
+      return KL_ERR_CUDA;
+    GemmParams gp{};
+    gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+    gp.tiles_n = static_cast<int>(cdiv(d, kBN));
+    gp.num_kb = static_cast<int>(cdiv(p->V, kBKe));
+    gp.m_fastest = 1;
+    gp.out = static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem);
+    gp.ld_out = d;
+    gp.rows_valid = static_cast<int>(Cn);
+    gp.cols_valid = static_cast<int>(d);
+    gp.status = &c.sc->status;
+    gp.spin_limit = spin_limit();
+    KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE>("gemm_dH", c.st, c.sms, ma, mb, gp,
+                                               2.0 * Cn * p->V * d)));
+  }
+  // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
+  {
+    CUtensorMap ma, mb;
+    const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * d * sizeof(Elem);
+    if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
+        !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe))
+      return KL_ERR_CUDA;
+    GemmParams gp{};
+    gp.tiles_m = static_cast<int>(cdiv(p->V, kBM));
+    gp.tiles_n = static_cast<int>(cdiv(d, kBN));
+    gp.num_kb = static_cast<int>(cdiv(Cn, kBKe));
+    gp.m_fastest = 0;
+    gp.out = dW;
+    gp.ld_out = d;
+    gp.rows_valid = static_cast<int>(p->V);
+    gp.cols_valid = static_cast<int>(d);
+    gp.beta = beta;
+    gp.status = &c.sc->status;
+    gp.spin_limit = spin_limit();
+    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM>("gemm_dW", c.st, c.sms, ma, mb, gp,
+                                               2.0 * Cn * p->V * d)));
+  }
+  return KL_OK;
+}
+
+int launch_count_valid(Ctx& c) {
+  LaunchScope ls("count_valid", c.st, 0, static_cast<double>(c.p->mask ? c.p->N : 0));
+  count_valid_kernel<<<1, 1024, 0, c.st>>>(c.p->mask, c.p->N, c.p->normalizer, c.sc);
+  return KL_LAUNCHED();
+}
+
+int launch_prep(Ctx& c, int64_t c0, int64_t Cn) {
+  const kl_problem* p = c.p;
+  const int K = p->K;
+  const int rows_per_block = 4;
+  const size_t smem = static_cast<size_t>(rows_per_block) * 3 * K * 4;
+  int* sidx = reinterpret_cast<int*>(c.ws + c.pl.off_sidx);
+  float* sq = reinterpret_cast<float*>(c.ws + c.pl.off_sq);
+  float2* rinfo = reinterpret_cast<float2*>(c.ws + c.pl.off_rinfo);
+  static bool attr[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev]) {
+    cudaFuncSetAttribute(prep_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         rows_per_block * 3 * kMaxK * 4);
+    attr[dev] = true;
+  }
+  LaunchScope ls("prep_topk", c.st, 0, static_cast<double>(Cn) * K * 16 + Cn * 12);
+  prep_topk_kernel<<<static_cast<unsigned>(cdiv(Cn, rows_per_block)), 32 * rows_per_block, smem,
+                     c.st>>>(p->topk_idx + c0 * K, p->topk_logit + c0 * K,
+                             p->teacher_lse ? p->teacher_lse + c0 : nullptr, c.invT,
+                             static_cast<int>(p->V), K, static_cast<int>(Cn), sidx, sq, rinfo,
+                             c.sc);
+  return KL_LAUNCHED();
+}
+
+int launch_row_reduce(Ctx& c, const float4* partials, int64_t c0, int64_t Cn, bool with_loss,
+                      float* lse_out, float* row_loss) {
+  const kl_problem* p = c.p;
+  const float2* rinfo =
+      with_loss ? reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo) : nullptr;
+  LaunchScope ls("row_reduce", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 16);
+  row_reduce_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
+      partials, c.pl.tiles_v, static_cast<int>(Cn), p->mask ? p->mask + c0 : nullptr, rinfo,
+      lse_out + c0, row_loss ? row_loss + c0 : nullptr);
+  return KL_LAUNCHED();
+}
+
+template <typename Elem>
+int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse,
+                        const float* g_dev, float g_host) {
+  const kl_problem* p = c.p;
+  static bool attr[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev]) {
+    cudaFuncSetAttribute(dlogits_topk_kernel<Elem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kMaxK * 4);
+    attr[dev] = true;
+  }
+  LaunchScope ls("dlogits_topk", c.st, 0, 2.0 * Cn * p->V * sizeof(Elem));
+  dlogits_topk_kernel<Elem><<<static_cast<unsigned>(Cn), 256, p->K * 4, c.st>>>(
+      S, c.pl.Vp, static_cast<int>(p->V), lse + c0, p->mask ? p->mask + c0 : nullptr,
+      reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
+      reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+      reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT);
+  return KL_LAUNCHED();
+}
+
+template <typename Elem>
+int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
+                        const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
+                        float* row_loss, int write_grad) {
+  const kl_problem* p = c.p;
+  LaunchScope ls("dlogits_full", c.st, 0,
+                 (write_grad ? 3.0 : 2.0) * Cn * p->V * sizeof(Elem));
+  dlogits_full_kernel<Elem><<<static_cast<unsigned>(Cn), 256, 0, c.st>>>(
+      S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
+      p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
+      row_loss ? row_loss + c0 : nullptr, write_grad);
+  return KL_LAUNCHED();
+}
+
+int launch_finalize(Ctx& c, const float* row_loss, float* loss) {
+  LaunchScope ls("finalize_loss", c.st, 0, static_cast<double>(c.p->N) * 4);
+  finalize_loss_kernel<<<1, 1024, 0, c.st>>>(row_loss, c.p->N, c.sc, loss);
+  return KL_LAUNCHED();
+}
+
+int launch_fill(Ctx& c, float* p, int64_t n, float v) {
+  if (n <= 0) return KL_OK;
+  LaunchScope ls("fill", c.st, 0, static_cast<double>(n) * 4);
+  fill_f32_kernel<<<static_cast<unsigned>(c.sms * 4), 256, 0, c.st>>>(p, n, v);
+  return KL_LAUNCHED();
+}
+
+int begin(const kl_problem* p, int entry, void* ws, size_t ws_bytes, void* stream, Ctx& c) {
+  KL_TRY(validate(p));
+  DevInfo di;
+  KL_TRY(current_device_info(&di));
+  c.p = p;
+  c.pl = make_plan(p, entry);
+  if (ws == nullptr) return KL_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return KL_ERR_ALIGN;
+  if (ws_bytes < c.pl.total) return KL_ERR_WORKSPACE;
+  c.ws = static_cast<uint8_t*>(ws);
+  c.sc = reinterpret_cast<Scalars*>(ws);
+  c.st = static_cast<cudaStream_t>(stream);
+  c.sms = di.sms;
+  c.invT = 1.0f / p->T;
+  return KL_OK;
+}
+
+// ------------------------------------------------------------------ entry bodies
+template <typename Elem>
+int run_fwd(Ctx& c, float* loss, float* lse_s, float* lse_t, float* row_loss) {
+  const kl_problem* p = c.p;
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(c.ws + c.pl.off_rl);
+  KL_TRY(launch_count_valid(c));
+  KL_TRY(prepare_heads(c));
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
+    const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
+    if (!c.pl.hidden) {
+      KL_TRY(launch_prep(c, c0, Cn));
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, nullptr, ps,
+                               reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+                               reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
+                               "gemm_logits_stats"));
+      KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
+    } else {
+      Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
+      Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
+      float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
+                               "gemm_logits_stats"));
+      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
+                               "gemm_teacher_logits"));
+      KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
+      KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, 0.f, rl, 0));
+    }
+  }
+  return launch_finalize(c, rl, loss);
+}
+
+template <typename Elem>
+int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
+            void* dH, float* dW, int accumulate) {
+  const kl_problem* p = c.p;
+  if (p->N == 0) return accumulate ? KL_OK : launch_fill(c, dW, p->V * p->d, 0.f);
+  Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
+  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
+  KL_TRY(launch_count_valid(c));
+  KL_TRY(prepare_heads(c));
+  if (sizeof(Elem) == 4)
+    KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
+                            reinterpret_cast<float*>(c.ws + c.pl.off_wT), c.pl.Vp, p->V, p->d));
+  for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
+    const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
+    if (!c.pl.hidden) {
+      KL_TRY(launch_prep(c, c0, Cn));
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, nullptr, nullptr, nullptr, 0,
+                               "gemm_logits_recompute"));
+      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
+    } else {
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, nullptr, nullptr, nullptr, 0,
+                               "gemm_logits_recompute"));
+      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, nullptr, nullptr, nullptr,
+                               0, "gemm_teacher_logits"));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, g_dev, g_host, nullptr,
+                                       1));
+    }
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
+  }
+  return KL_OK;
+}
+
+template <typename Elem>
+int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* dW,
+                int accumulate) {
+  const kl_problem* p = c.p;
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(c.ws + c.pl.off_rl);
+  float* lse_s = reinterpret_cast<float*>(c.ws + c.pl.off_lse_s);
+  float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
+  Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
+  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+  KL_TRY(launch_count_valid(c));
+  if (p->N == 0) {
+    if (!accumulate) KL_TRY(launch_fill(c, dW, p->V * p->d, 0.f));
+    return launch_finalize(c, rl, loss);
+  }
+  KL_TRY(prepare_heads(c));
+  if (sizeof(Elem) == 4)
+    KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
+                            reinterpret_cast<float*>(c.ws + c.pl.off_wT), c.pl.Vp, p->V, p->d));
+  for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
+    const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
+    if (!c.pl.hidden) {
+      KL_TRY(launch_prep(c, c0, Cn));
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps,
+                               reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+                               reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
+                               "gemm_logits_stats"));
+      KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
+      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g));
+    } else {
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
+                               "gemm_logits_stats"));
+      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
+                               "gemm_teacher_logits"));
+      KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
+      KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1));
+    }
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
+  }
+  return launch_finalize(c, rl, loss);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+size_t kl_workspace_bytes(const kl_problem* p, int entry) {
+  if (validate_shape(p) != KL_OK || entry < KL_ENTRY_FWD || entry > KL_ENTRY_FWD_BWD) return 0;
+  return make_plan(p, entry).total;
+}
+
+int kl_fwd(const kl_problem* p, void* ws, size_t ws_bytes, float* loss, float* lse_s,
+           float* lse_t, float* row_loss, void* stream) {
+  Ctx c;
+  KL_TRY(begin(p, KL_ENTRY_FWD, ws, ws_bytes, stream, c));
+  if (loss == nullptr || (p->N > 0 && lse_s == nullptr) ||
+      (p->N > 0 && p->teacher == KL_TEACHER_HIDDEN && lse_t == nullptr))
+    return KL_ERR_NULL;
+  return p->dtype == KL_DTYPE_BF16 ? run_fwd<__nv_bfloat16>(c, loss, lse_s, lse_t, row_loss)
+                                   : run_fwd<float>(c, loss, lse_s, lse_t, row_loss);
+}
+
+int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,
+           const float* lse_t, const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+           void* stream) {
+  Ctx c;
+  KL_TRY(begin(p, KL_ENTRY_BWD, ws, ws_bytes, stream, c));
+  if (dW == nullptr || grad_loss == nullptr ||
+      (p->N > 0 && (dH == nullptr || lse_s == nullptr)) ||
+      (p->N > 0 && p->teacher == KL_TEACHER_HIDDEN && lse_t == nullptr))
+    return KL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(dH) | reinterpret_cast<uintptr_t>(dW)) & 15)
+    return KL_ERR_ALIGN;
+  return p->dtype == KL_DTYPE_BF16
+             ? run_bwd<__nv_bfloat16>(c, lse_s, lse_t, grad_loss, 0.f, dH, dW, accumulate_dW)
+             : run_bwd<float>(c, lse_s, lse_t, grad_loss, 0.f, dH, dW, accumulate_dW);
+}
+
+int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss, float* loss,
+               float* row_loss, void* dH, float* dW, int accumulate_dW, void* stream) {
+  Ctx c;
+  KL_TRY(begin(p, KL_ENTRY_FWD_BWD, ws, ws_bytes, stream, c));
+  if (loss == nullptr || dW == nullptr || (p->N > 0 && dH == nullptr)) return KL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(dH) | reinterpret_cast<uintptr_t>(dW)) & 15)
+    return KL_ERR_ALIGN;
+  return p->dtype == KL_DTYPE_BF16
+             ? run_fwd_bwd<__nv_bfloat16>(c, grad_loss, loss, row_loss, dH, dW, accumulate_dW)
+             : run_fwd_bwd<float>(c, grad_loss, loss, row_loss, dH, dW, accumulate_dW);
+}
+
+int kl_status(void* ws, void* stream) {
+  if (ws == nullptr) return KL_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KL_ERR_CUDA;
+  int s = 0;
+  if (cudaMemcpy(&s, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KL_ERR_CUDA;
+  return s;
+}
+
+const char* kl_status_string(int code) {
+  switch (code) {
+    case KL_OK: return "ok";
+    case KL_ERR_NULL: return "a required pointer is NULL";
+    case KL_ERR_SHAPE: return "a size is out of range";
+    case KL_ERR_DTYPE: return "unknown dtype or teacher mode";
+    case KL_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case KL_ERR_WORKSPACE: return "workspace smaller than kl_workspace_bytes()";
+    case KL_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case KL_ERR_INDEX: return "top-K cache index out of range or duplicated";
+    case KL_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case KL_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200-class)";
+    case KL_ERR_ARG: return "bad argument (temperature, chunk size or normaliser)";
+    default: return "unknown status";
+  }
+}
+
+uint64_t kl_launch_count(void) { return g_launches.load(); }
+
+int kl_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& k : g_prof)
+    for (auto& e : k.ev) {
+      g_ev_pool.push_back(e.first);
+      g_ev_pool.push_back(e.second);
+    }
+  g_prof.clear();
+  g_prof.reserve(64);
+  g_prof_on = true;
+  return KL_OK;
+}
+
+int kl_profile_end(kl_profile_entry* out, int max_entries) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  int n = 0;
+  for (auto& k : g_prof) {
+    double ms = 0;
+    for (auto& e : k.ev) {
+      if (cudaEventSynchronize(e.second) != cudaSuccess) return -KL_ERR_CUDA;
+      float t = 0;
+      if (cudaEventElapsedTime(&t, e.first, e.second) != cudaSuccess) return -KL_ERR_CUDA;
+      ms += t;
+    }
+    if (out != nullptr && n < max_entries) {
+      kl_profile_entry& o = out[n];
+      memset(&o, 0, sizeof(o));
+      strncpy(o.name, k.name.c_str(), sizeof(o.name) - 1);
+      o.launches = k.launches;
+      o.total_ms = ms;
+      o.flops = k.flops;
+      o.bytes = k.bytes;
+    }
+    ++n;
+  }
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,436 @@
+// kl_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for the three
+// contractions of the fused KL loss, with the loss arithmetic fused into the
+// epilogue ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits
+// and a Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection
+// is integrated into the loss and each logit chunk is transient).
+//
+//   C[M, N] = A[M, K] . B[N, K]^T   (bf16 -> kind::f16, fp32 -> kind::tf32;
+//                                     fp32 accumulation in TMEM)
+//
+//   EPI_STATS  logits tile S = H_c . W^T: per (row, 256-column tile) the
+//              online max and sum of 2^(s~ log2 e) and the cross term
+//              sum_i q_i s~_{idx_i} of the cached top-K entries that fall in
+//              the tile (gathered from the fp32 accumulator); optionally
+//              stores s~ = s / T to the chunk's logit buffer.
+//   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
+//   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, read-modify-write across chunks.
+//
+// Roles (192 threads, one CTA per SM, grid-strided over output tiles):
+//   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
+//              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
+//   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
+//   warp 5     TMEM allocator + MMA issuer (one thread).
+// Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
+// i overlap the main loop of tile i + 1.
+//
+// Every wait on an mbarrier is bounded (spin_limit clock cycles); when one
+// runs out the CTA records KL_ERR_TIMEOUT in *status, every role leaves its
+// loop, in-flight copies and MMAs are drained (again with a bound) and TMEM is
+// released before the CTA exits.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "kl_ptx.cuh"
+
+namespace ckl {
+
+constexpr int kBM = 128;          // tile rows (TMEM lanes)
+constexpr int kBN = 256;          // tile columns (TMEM columns per accumulator)
+constexpr int kStages = 4;        // smem ring depth
+constexpr int kRowBytes = 128;    // one 128-B swizzle span per tile row / slab row
+constexpr int kATileBytes = kBM * kRowBytes;
+constexpr int kBTileBytes = kBN * kRowBytes;
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 2 * kBN;
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2 };
+
+struct GemmParams {
+  int tiles_m, tiles_n, num_kb;
+  int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
+  void* out;           // STATS: logit buffer (nullable); STORE: dH; ACCUM: dW
+  int64_t ld_out;      // row stride of out, elements
+  int rows_valid;      // output rows that exist (M extent)
+  int cols_valid;      // output columns that exist (N extent)
+  int cols_store;      // STATS: columns written to the logit buffer (padded V)
+  float scale;         // STATS: 1 / T
+  int beta;            // ACCUM: 0 overwrite, 1 accumulate
+  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross, 0)
+  const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
+  const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
+  int ktop;            // STATS gather: entries per row (0 = no gather)
+  int* status;         // device status word
+  long long spin_limit;
+};
+
+struct Ctl {
+  int* status;
+  long long limit;
+  volatile int* abort_flag;
+};
+
+// Bounded wait for the phase of the given parity; false when the CTA aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*c.abort_flag) return false;
+    if (clock64() - t0 > c.limit) {
+      *c.abort_flag = 1;
+      atomicCAS(c.status, 0, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <typename Elem>
+struct ElemTraits;
+template <>
+struct ElemTraits<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr uint32_t kFmt = 1;  // bf16
+};
+template <>
+struct ElemTraits<float> {
+  static constexpr int kBytes = 4;
+  static constexpr uint32_t kFmt = 2;  // tf32
+};
+
+__device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm, int& tn) {
+  if (p.m_fastest) {
+    tm = t % p.tiles_m;
+    tn = t / p.tiles_m;
+  } else {
+    tn = t % p.tiles_n;
+    tm = t / p.tiles_n;
+  }
+}
+
+// Pack 8 consecutive fp32 values into one 16-byte vector of Elem.
+template <typename Elem>
+__device__ __forceinline__ void store_vec(Elem* dst, const float* v);
+template <>
+__device__ __forceinline__ void store_vec<__nv_bfloat16>(__nv_bfloat16* dst, const float* v) {
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+  __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
+  __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
+  uint4 u;
+  u.x = *reinterpret_cast<uint32_t*>(&h0);
+  u.y = *reinterpret_cast<uint32_t*>(&h1);
+  u.z = *reinterpret_cast<uint32_t*>(&h2);
+  u.w = *reinterpret_cast<uint32_t*>(&h3);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <typename Elem, int A_MN, int B_MN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int kEB = ElemTraits<Elem>::kBytes;
+  constexpr int kBKe = kRowBytes / kEB;       // K elements per stage (64 / 32)
+  constexpr int kUmmaK = 32 / kEB;            // K per MMA instruction (16 / 8)
+  constexpr int kKSteps = kBKe / kUmmaK;      // 4
+  constexpr int kMNe = kRowBytes / kEB;       // MN elements per MN-major slab
+  constexpr int kSlabBytes = kBKe * kRowBytes;
+  constexpr uint32_t kIdesc = idesc_dense(ElemTraits<Elem>::kFmt, kBM, kBN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty_bar = full_bar + kStages;
+  uint64_t* tfull_bar = empty_bar + kStages;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int total_tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 4 * 32);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const Ctl ctl{p.status, p.spin_limit, abort_flag};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, p, tm, tn);
+        const int m0 = tm * kBM, n0 = tn * kBN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          const uint32_t s = issued % kStages;
+          const uint32_t ph = (issued / kStages) & 1u;
+          if (!wait_bar(&empty_bar[s], ph ^ 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_s = smem + s * kStageBytes;
+          uint8_t* b_s = a_s + kATileBytes;
+          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+          const int k0 = kb * kBKe;
+          if (A_MN) {
+#pragma unroll
+            for (int sl = 0; sl < kBM / kMNe; ++sl)
+              tma_load_2d(&tmA, &full_bar[s], a_s + sl * kSlabBytes, m0 + sl * kMNe, k0);
+          } else {
+            tma_load_2d(&tmA, &full_bar[s], a_s, k0, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int sl = 0; sl < kBN / kMNe; ++sl)
+              tma_load_2d(&tmB, &full_bar[s], b_s + sl * kSlabBytes, n0 + sl * kMNe, k0);
+          } else {
+            tma_load_2d(&tmB, &full_bar[s], b_s, k0, n0);
+          }
+          ++issued;
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA exits.
+        Ctl drain{p.status, p.spin_limit, abort_flag};
+        volatile int no_abort = 0;
+        drain.abort_flag = &no_abort;
+        const uint32_t first = issued > kStages ? issued - kStages : 0;
+        for (uint32_t n = first; n < issued; ++n)
+          wait_bar(&full_bar[n % kStages], (n / kStages) & 1u, drain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t consumed = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+        const uint32_t buf = local & 1u;
+        const uint32_t aph = (local >> 1) & 1u;
+        if (!wait_bar(&tempty_bar[buf], aph ^ 1u, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * kBN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          const uint32_t s = consumed % kStages;
+          const uint32_t ph = (consumed / kStages) & 1u;
+          if (!wait_bar(&full_bar[s], ph, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int j = 0; j < kKSteps; ++j) {
+            const uint64_t ad = A_MN ? sdesc_sw128(a_addr + j * (kUmmaK / 8) * 1024,
+                                                   kSlabBytes, 1024)
+                                     : sdesc_sw128(a_addr + j * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(b_addr + j * (kUmmaK / 8) * 1024,
+                                                   kSlabBytes, 1024)
+                                     : sdesc_sw128(b_addr + j * 32, 16, 1024);
+            if (kEB == 2)
+              umma_f16(d_tmem, ad, bd, kIdesc, (kb | j) != 0);
+            else
+              umma_tf32(d_tmem, ad, bd, kIdesc, (kb | j) != 0);
+          }
+          umma_commit(&empty_bar[s]);  // frees the smem stage when these MMAs finish
+          ++consumed;
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[buf]);  // accumulator ready for the epilogue
+      }
+      if (!ok) {
+        // Wait (bounded) for every MMA already issued before TMEM is released.
+        volatile int no_abort = 0;
+        Ctl drain{p.status, p.spin_limit, &no_abort};
+        umma_commit(drain_bar);
+        wait_bar(drain_bar, 0, drain);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int r = warp * 32 + lane;  // accumulator row owned by this thread
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    uint32_t local = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+      int tm, tn;
+      tile_coords(t, p, tm, tn);
+      const uint32_t buf = local & 1u;
+      const uint32_t aph = (local >> 1) & 1u;
+      if (!wait_bar(&tfull_bar[buf], aph, ctl)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_base + buf * kBN;
+      const int grow = tm * kBM + r;
+      const bool rv = grow < p.rows_valid;
+      const int col0 = tn * kBN;
+
+      if (EPI == EPI_STATS) {
+        const float s2 = p.scale * kLog2e;
+        float mx = -INFINITY, se = 0.f, cross = 0.f;
+        int gi = 0, gcol = 0x7fffffff;
+        const int* ri = nullptr;
+        const float* rq = nullptr;
+        if (p.ktop > 0 && rv) {
+          ri = p.sidx + static_cast<int64_t>(grow) * p.ktop;
+          rq = p.sq + static_cast<int64_t>(grow) * p.ktop;
+          int lo = 0, hi = p.ktop;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(ri + mid) < col0) lo = mid + 1; else hi = mid;
+          }
+          gi = lo;
+          gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
+        }
+        Elem* orow = (p.out != nullptr && rv)
+                         ? static_cast<Elem*>(p.out) + static_cast<int64_t>(grow) * p.ld_out
+                         : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (c == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty_bar[buf]);
+          }
+          const int cb = col0 + c * 32;
+          const int nvalid = p.cols_valid - cb;  // columns < V in this slab
+          float cm = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(v[i]) * s2;
+            cm = fmaxf(cm, i < nvalid ? x : -INFINITY);
+          }
+          if (cm > -INFINITY) {
+            const float nm = fmaxf(mx, cm);
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(v[i]) * s2;
+              acc += i < nvalid ? ex2_approx(x - nm) : 0.f;
+            }
+            se = se * ex2_approx(mx - nm) + acc;
+            mx = nm;
+          }
+          while (gcol < cb + 32) {  // cached entries inside this 32-column slab
+            const int k = gcol - cb;
+            float val = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) val = (i == k) ? __uint_as_float(v[i]) : val;
+            cross += __ldg(rq + gi) * (val * p.scale);
+            ++gi;
+            gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
+          }
+          if (orow != nullptr) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (cb + g * 8 < p.cols_store) {
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[g * 8 + i]) * p.scale;
+                store_vec<Elem>(orow + cb + g * 8, f);
+              }
+            }
+          }
+        }
+        if (rv && p.partials != nullptr)
+          p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (c == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty_bar[buf]);
+          }
+          if (!rv) continue;
+          const int cb = col0 + c * 32;
+          if (EPI == EPI_STORE) {
+            Elem* orow = static_cast<Elem*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (cb + g * 8 < p.cols_valid) {
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[g * 8 + i]);
+                store_vec<Elem>(orow + cb + g * 8, f);
+              }
+            }
+          } else {  // EPI_ACCUM, fp32 out
+            float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              if (cb + g * 4 < p.cols_valid) {
+                float4* o = reinterpret_cast<float4*>(orow + cb + g * 4);
+                float4 a = make_float4(__uint_as_float(v[g * 4 + 0]), __uint_as_float(v[g * 4 + 1]),
+                                       __uint_as_float(v[g * 4 + 2]), __uint_as_float(v[g * 4 + 3]));
+                if (p.beta) {
+                  const float4 old = *o;
+                  a.x += old.x;
+                  a.y += old.y;
+                  a.z += old.z;
+                  a.w += old.w;
+                }
+                *o = a;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace ckl

@@ -1,0 +1,403 @@
+// kl_rowops.cuh -- the SIMT (HBM-bound) steps of the fused KL loss.
+//
+// Source: "Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and
+// a Fused Chunked KL Loss", §3 "Offline distillation" (teacher-entropy, cross
+// and mass terms need only the cached support; log Z is the one full-vocabulary
+// reduction) and §3 "Offline implementations" (each chunk writes its scalar
+// log Z values and scatters over the K retained entries); KDFlow abstract for
+// the teacher-hidden mode.
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kl_ptx.cuh"
+
+namespace ckl {
+
+constexpr int kStatusIndex = 7;  // KL_ERR_INDEX
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kEmpty = 0x7fffffff;  // sorted-cache sentinel for an empty slot
+
+// Scalars at the head of the workspace.
+struct Scalars {
+  int status;     // KL_OK or a device-detected error
+  int n_valid;    // rows with mask = 1
+  float norm;     // divisor of the loss mean (caller's normaliser or n_valid)
+  float pad;
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Round-to-nearest onto the tf32 grid (10 explicit mantissa bits).  The
+// tensor cores read only those bits of an fp32 operand and drop the rest, which
+// biases every product towards zero; operands of the fp32 path are rounded
+// first so the error is unbiased.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+// Value as it will be stored in an operand buffer of element type Elem.
+template <typename Elem>
+__device__ __forceinline__ float operand_round(float x) {
+  return sizeof(Elem) == 4 ? round_tf32(x) : x;
+}
+
+template <typename Elem>
+__device__ __forceinline__ float to_f(Elem x);
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <>
+__device__ __forceinline__ float to_f<float>(float x) {
+  return x;
+}
+template <typename Elem>
+__device__ __forceinline__ Elem from_f(float x);
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ float from_f<float>(float x) {
+  return x;
+}
+
+// Load / store 8 consecutive elements as one or two 16-byte vectors.
+template <typename Elem>
+__device__ __forceinline__ void load8(const Elem* src, float* f);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* src, float* f) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* src, float* f) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0];
+  const float4 b = reinterpret_cast<const float4*>(src)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+template <typename Elem>
+__device__ __forceinline__ void store8(Elem* dst, const float* f);
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* dst, const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <>
+__device__ __forceinline__ void store8<float>(float* dst, const float* f) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// Resets the status word and counts the rows that enter the mean.
+__global__ void count_valid_kernel(const uint8_t* mask, int64_t N, float normalizer,
+                                   Scalars* sc) {
+  __shared__ int part[32];
+  int c = 0;
+  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) c += mask ? (mask[i] != 0) : 1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
+    sc->status = 0;
+    sc->n_valid = tot;
+    sc->norm = normalizer > 0.f ? normalizer : static_cast<float>(tot);
+  }
+}
+
+// Per cached row (one warp per row): validate ids, sort the K entries by
+// vocabulary id (empty slots last, as kEmpty), and turn teacher logits into
+// probabilities on the support:
+//   partial mass (lse_t != nullptr): q = exp(t / T - lse_t)
+//   renormalised:                    q = softmax over valid entries of t / T
+// rowinfo = (m = sum q, sum q log q).
+__global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
+                                 const float* __restrict__ logit,
+                                 const float* __restrict__ lse_t, float invT, int V, int K,
+                                 int rows, int* __restrict__ sidx, float* __restrict__ sq,
+                                 float2* __restrict__ rowinfo, Scalars* sc) {
+  extern __shared__ int prep_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  int* key = prep_smem + warp * 3 * K;
+  float* tv = reinterpret_cast<float*>(key + K);
+  float* qv = tv + K;
+  const int32_t* ri = idx + static_cast<int64_t>(row) * K;
+  const float* rl = logit + static_cast<int64_t>(row) * K;
+  bool bad = false;
+  float tmax = -INFINITY;
+  for (int i = lane; i < K; i += 32) {
+    int k = ri[i];
+    if (k < -1 || k >= V) {
+      bad = true;
+      k = -1;
+    }
+    key[i] = k < 0 ? kEmpty : k;
+    const float t = rl[i] * invT;
+    tv[i] = t;
+    if (k >= 0) tmax = fmaxf(tmax, t);
+  }
+  __syncwarp();
+  float m = 0.f, negent = 0.f;
+  if (lse_t != nullptr) {
+    const float l = lse_t[row];
+    for (int i = lane; i < K; i += 32) {
+      const float q = key[i] != kEmpty ? expf(tv[i] - l) : 0.f;
+      qv[i] = q;
+      m += q;
+      negent += q > 0.f ? q * logf(q) : 0.f;
+    }
+  } else {
+    tmax = warp_max(tmax);
+    float z = 0.f;
+    for (int i = lane; i < K; i += 32) z += key[i] != kEmpty ? expf(tv[i] - tmax) : 0.f;
+    z = warp_sum(z);
+    const float lz = logf(z);
+    for (int i = lane; i < K; i += 32) {
+      const bool ok = key[i] != kEmpty && z > 0.f;
+      const float q = ok ? expf(tv[i] - tmax) / z : 0.f;
+      qv[i] = q;
+      m += q;
+      negent += (ok && q > 0.f) ? q * (tv[i] - tmax - lz) : 0.f;
+    }
+  }
+  __syncwarp();
+  m = warp_sum(m);
+  negent = warp_sum(negent);
+  int* so = sidx + static_cast<int64_t>(row) * K;
+  float* qo = sq + static_cast<int64_t>(row) * K;
+  for (int i = lane; i < K; i += 32) {
+    const int ki = key[i];
+    int rank = 0;
+    for (int j = 0; j < K; ++j) {
+      const int kj = key[j];
+      rank += (kj < ki) || (kj == ki && j < i);
+      bad |= (kj == ki && j != i && ki != kEmpty);
+    }
+    so[rank] = ki;
+    qo[rank] = qv[i];
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(&sc->status, 0, kStatusIndex);
+  if (lane == 0) rowinfo[row] = make_float2(m, negent);
+}
+
+// Split-V merge (one warp per row): partials (max2, sumexp2, cross) of every
+// 256-column tile -> lse = ln 2 * (M + log2 Z).  In top-K mode also the row
+// loss l = [sum q log q] - [sum q s~] + m * lse (0 on masked rows).
+__global__ void row_reduce_kernel(const float4* __restrict__ partials, int tiles_n, int rows,
+                                  const uint8_t* __restrict__ mask,
+                                  const float2* __restrict__ rowinfo, float* __restrict__ lse_out,
+                                  float* __restrict__ row_loss) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const float4* pr = partials + static_cast<int64_t>(row) * tiles_n;
+  float M = -INFINITY;
+  for (int i = lane; i < tiles_n; i += 32) M = fmaxf(M, pr[i].x);
+  M = warp_max(M);
+  float Z = 0.f, cross = 0.f;
+  for (int i = lane; i < tiles_n; i += 32) {
+    const float4 v = pr[i];
+    Z += v.y * ex2_approx(v.x - M);
+    cross += v.z;
+  }
+  Z = warp_sum(Z);
+  cross = warp_sum(cross);
+  if (lane == 0) {
+    const float lse = (M + log2f(Z)) * kLn2;
+    lse_out[row] = lse;
+    if (rowinfo != nullptr && row_loss != nullptr) {
+      const bool keep = mask == nullptr || mask[row] != 0;
+      const float2 ri = rowinfo[row];
+      row_loss[row] = keep ? (ri.y - cross + ri.x * lse) : 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ float grad_coef(const uint8_t* mask, int row, const Scalars* sc,
+                                           const float* g_dev, float g_host, float invT) {
+  const bool keep = mask == nullptr || mask[row] != 0;
+  const float g = g_dev != nullptr ? *g_dev : g_host;
+  const float norm = sc->norm;
+  return (keep && norm > 0.f) ? g / norm * invT : 0.f;
+}
+
+// dS for the top-K loss, in place over the chunk's logit buffer (one CTA per
+// row):  dS_j = c (m p_s,j - q_j [j in S]),  c = g / (n T),  p_s = exp(s~ - lse).
+// The K cached positions are read before the dense pass and rewritten after it.
+template <typename Elem>
+__global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
+                                    const float* __restrict__ lse, const uint8_t* __restrict__ mask,
+                                    const float2* __restrict__ rowinfo,
+                                    const int* __restrict__ sidx, const float* __restrict__ sq,
+                                    int K, const Scalars* sc, const float* g_dev, float g_host,
+                                    float invT) {
+  extern __shared__ float sval[];
+  const int row = blockIdx.x;
+  Elem* srow = S + static_cast<int64_t>(row) * ld;
+  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT);
+  const int nvec = (V + 7) >> 3;
+  if (coef == 0.f) {
+    const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) store8<Elem>(srow + v * 8, z);
+    return;
+  }
+  const int* ri = sidx + static_cast<int64_t>(row) * K;
+  const float* rq = sq + static_cast<int64_t>(row) * K;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    const int j = ri[i];
+    sval[i] = j != kEmpty ? to_f<Elem>(srow[j]) : 0.f;
+  }
+  __syncthreads();
+  const float m = rowinfo[row].x;
+  const float l2 = lse[row] * kLog2e;
+  const float cm = coef * m;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float f[8];
+    load8<Elem>(srow + v * 8, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      f[i] = (v * 8 + i < V) ? operand_round<Elem>(cm * ex2_approx(fmaf(f[i], kLog2e, -l2)))
+                             : 0.f;
+    store8<Elem>(srow + v * 8, f);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    const int j = ri[i];
+    if (j != kEmpty)
+      srow[j] = from_f<Elem>(
+          operand_round<Elem>(coef * (m * ex2_approx(fmaf(sval[i], kLog2e, -l2)) - rq[i])));
+  }
+}
+
+// Full-vocabulary mode (one CTA per row): A = sum_j p_t,j (t~_j - s~_j) so that
+// l = A - lse_t + lse_s; optionally dS = c (p_s - p_t) in place over S.
+template <typename Elem>
+__global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict__ Tt, int64_t ld,
+                                    int V, const float* __restrict__ lse_s,
+                                    const float* __restrict__ lse_t,
+                                    const uint8_t* __restrict__ mask, const Scalars* sc,
+                                    const float* g_dev, float g_host, float invT,
+                                    float* __restrict__ row_loss, int write_grad) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  Elem* srow = S + static_cast<int64_t>(row) * ld;
+  const Elem* trow = Tt + static_cast<int64_t>(row) * ld;
+  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT);
+  const float ls2 = lse_s[row] * kLog2e, lt2 = lse_t[row] * kLog2e;
+  const int nvec = (V + 7) >> 3;
+  float A = 0.f;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float fs[8], ft[8];
+    load8<Elem>(srow + v * 8, fs);
+    load8<Elem>(trow + v * 8, ft);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = v * 8 + i < V;
+      const float pt = ex2_approx(fmaf(ft[i], kLog2e, -lt2));
+      const float ps = ex2_approx(fmaf(fs[i], kLog2e, -ls2));
+      A += in ? pt * (ft[i] - fs[i]) : 0.f;
+      fs[i] = in ? operand_round<Elem>(coef * (ps - pt)) : 0.f;
+    }
+    if (write_grad) store8<Elem>(srow + v * 8, fs);
+  }
+  A = warp_sum(A);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = A;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    a = warp_sum(a);
+    if (threadIdx.x == 0 && row_loss != nullptr) {
+      const bool keep = mask == nullptr || mask[row] != 0;
+      row_loss[row] = keep ? a - lse_t[row] + lse_s[row] : 0.f;
+    }
+  }
+}
+
+// loss = sum_n row_loss[n] / norm, summed in fp64 in a fixed order.
+__global__ void finalize_loss_kernel(const float* __restrict__ row_loss, int64_t N,
+                                     const Scalars* sc, float* loss) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) s += row_loss[i];
+  s = warp_sum_d(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+    a = warp_sum_d(a);
+    if (threadIdx.x == 0) *loss = sc->norm > 0.f ? static_cast<float>(a / sc->norm) : 0.f;
+  }
+}
+
+// dst[c][r] = tf32-rounded src[r][c] for a rows x cols fp32 block (32 x 32
+// smem tiles).  tf32 operands are kept K-major: the 128-byte swizzle does not
+// serve MN-major 32-bit operands, so the fp32 path transposes them instead.
+__global__ void transpose_f32_kernel(const float* __restrict__ src, int64_t ld_src,
+                                     float* __restrict__ dst, int64_t ld_dst, int rows,
+                                     int cols) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < rows && c < cols) ? src[static_cast<int64_t>(r) * ld_src + c] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < cols && r < rows)
+      dst[static_cast<int64_t>(c) * ld_dst + r] = round_tf32(tile[threadIdx.x][i]);
+  }
+}
+
+// dst = tf32-rounded src for `rows` rows of `cols` fp32 values (row strides
+// ld_src, ld_dst).
+__global__ void round_tf32_kernel(const float* __restrict__ src, int64_t ld_src,
+                                  float* __restrict__ dst, int64_t ld_dst, int64_t rows,
+                                  int64_t cols) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / cols, c = i - r * cols;
+    dst[r * ld_dst + c] = round_tf32(src[r * ld_src + c]);
+  }
+}
+
+__global__ void fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
+}  // namespace ckl

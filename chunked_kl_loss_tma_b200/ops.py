@@ -1,0 +1,183 @@
+"""Torch-facing calls of the fused, chunked distillation KL loss.
+
+PyTorch supplies device memory and the current stream; every step of the loss
+runs in libchunkedkl.so through its C ABI (see include/chunked_kl.h for what
+each call computes, argument layouts and error behaviour).
+
+    out = kl_fwd_bwd(H, W, topk_idx=idx, topk_logit=val, teacher_lse=lse, T=1.0)
+    out["loss"], out["dH"], out["dW"]
+
+    loss = fused_kl_loss(H, W, topk_idx=idx, topk_logit=val)   # autograd
+    loss.backward()                                            # H.grad, W.grad
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+_DT = {torch.bfloat16: L.KL_DTYPE_BF16, torch.float32: L.KL_DTYPE_F32}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, name, dtype=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
+                 Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0):
+    """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive)."""
+    if not isinstance(H, torch.Tensor) or not H.is_cuda:
+        raise ValueError("H must be a CUDA tensor")
+    dev = H.device
+    if H.dtype not in _DT:
+        raise TypeError("H must be bfloat16 or float32")
+    _need(H, "H", H.dtype, dev)
+    _need(W, "W", H.dtype, dev)
+    if H.dim() != 2 or W.dim() != 2 or H.shape[1] != W.shape[1]:
+        raise ValueError("H must be [N, d] and W [V, d]")
+    if mask is not None and mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    _need(mask, "mask", torch.uint8, dev)
+    p = L.KLProblem()
+    p.N, p.d = H.shape
+    p.V = W.shape[0]
+    p.dtype = _DT[H.dtype]
+    p.H, p.W, p.mask = _ptr(H), _ptr(W), _ptr(mask)
+    p.T = float(T)
+    p.chunk_tokens = int(chunk_tokens)
+    p.normalizer = float(normalizer)
+    keep = [H, W, mask]
+    if Ht is not None:
+        _need(Ht, "Ht", H.dtype, dev)
+        _need(Wt, "Wt", H.dtype, dev)
+        if Ht.shape[0] != H.shape[0] or Wt.shape[0] != W.shape[0] or Ht.shape[1] != Wt.shape[1]:
+            raise ValueError("Ht must be [N, d_t] and Wt [V, d_t]")
+        p.teacher = L.KL_TEACHER_HIDDEN
+        p.d_t = Ht.shape[1]
+        p.Ht, p.Wt = _ptr(Ht), _ptr(Wt)
+        keep += [Ht, Wt]
+    else:
+        if topk_idx is None or topk_logit is None:
+            raise ValueError("give either topk_idx/topk_logit or Ht/Wt")
+        _need(topk_idx, "topk_idx", torch.int32, dev)
+        _need(topk_logit, "topk_logit", torch.float32, dev)
+        _need(teacher_lse, "teacher_lse", torch.float32, dev)
+        if topk_idx.shape != topk_logit.shape or topk_idx.shape[0] != H.shape[0]:
+            raise ValueError("topk_idx and topk_logit must both be [N, K]")
+        p.teacher = L.KL_TEACHER_TOPK
+        p.K = topk_idx.shape[1]
+        p.topk_idx, p.topk_logit, p.teacher_lse = (_ptr(topk_idx), _ptr(topk_logit),
+                                                   _ptr(teacher_lse))
+        keep += [topk_idx, topk_logit, teacher_lse]
+    return p, keep
+
+
+def workspace_bytes(problem, entry):
+    n = L.kl_workspace_bytes(problem, entry)
+    if n == 0:
+        raise ValueError("invalid problem (kl_workspace_bytes returned 0)")
+    return n
+
+
+def alloc_workspace(problem, entry, device):
+    return torch.empty(workspace_bytes(problem, entry), dtype=torch.uint8, device=device)
+
+
+def _stream(device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def kl_fwd_bwd(H, W, *, grad_loss=1.0, dW=None, accumulate_dW=False, want_row_loss=False,
+               workspace=None, **kw):
+    """Fused forward + backward.  Returns dict(loss, row_loss, dH, dW)."""
+    p, keep = make_problem(H, W, **kw)
+    dev = H.device
+    ws = workspace if workspace is not None else alloc_workspace(p, L.KL_ENTRY_FWD_BWD, dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    row_loss = torch.empty(H.shape[0], dtype=torch.float32, device=dev) if want_row_loss else None
+    dH = torch.empty_like(H)
+    if dW is None:
+        dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+        accumulate_dW = False
+    _need(dW, "dW", torch.float32, dev)
+    L.check(L.kl_fwd_bwd(p, ws.data_ptr(), ws.numel(), grad_loss, loss.data_ptr(),
+                         _ptr(row_loss), dH.data_ptr(), dW.data_ptr(), accumulate_dW,
+                         _stream(dev)), "kl_fwd_bwd")
+    return dict(loss=loss, row_loss=row_loss, dH=dH, dW=dW, workspace=ws)
+
+
+def kl_fwd(H, W, *, workspace=None, want_row_loss=True, **kw):
+    """Forward only.  Returns dict(loss, lse_s, lse_t, row_loss)."""
+    p, keep = make_problem(H, W, **kw)
+    dev = H.device
+    ws = workspace if workspace is not None else alloc_workspace(p, L.KL_ENTRY_FWD, dev)
+    N = H.shape[0]
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse_s = torch.empty(N, dtype=torch.float32, device=dev)
+    lse_t = torch.empty(N, dtype=torch.float32, device=dev) if kw.get("Ht") is not None else None
+    row_loss = torch.empty(N, dtype=torch.float32, device=dev) if want_row_loss else None
+    L.check(L.kl_fwd(p, ws.data_ptr(), ws.numel(), loss.data_ptr(), lse_s.data_ptr(),
+                     _ptr(lse_t), _ptr(row_loss), _stream(dev)), "kl_fwd")
+    return dict(loss=loss, lse_s=lse_s, lse_t=lse_t, row_loss=row_loss, workspace=ws)
+
+
+def kl_bwd(H, W, lse_s, lse_t=None, *, grad_loss=None, dW=None, accumulate_dW=False,
+           workspace=None, **kw):
+    """Backward with logits recomputed per chunk.  grad_loss: device scalar
+    tensor (default 1).  Returns dict(dH, dW)."""
+    p, keep = make_problem(H, W, **kw)
+    dev = H.device
+    ws = workspace if workspace is not None else alloc_workspace(p, L.KL_ENTRY_BWD, dev)
+    if grad_loss is None:
+        grad_loss = torch.ones((), dtype=torch.float32, device=dev)
+    grad_loss = _need(grad_loss.to(torch.float32).contiguous(), "grad_loss", torch.float32, dev)
+    dH = torch.empty_like(H)
+    if dW is None:
+        dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+        accumulate_dW = False
+    L.check(L.kl_bwd(p, ws.data_ptr(), ws.numel(), lse_s.data_ptr(), _ptr(lse_t),
+                     grad_loss.data_ptr(), dH.data_ptr(), dW.data_ptr(), accumulate_dW,
+                     _stream(dev)), "kl_bwd")
+    return dict(dH=dH, dW=dW, workspace=ws)
+
+
+def status(workspace):
+    """Synchronise and return the device-side status word of a workspace."""
+    return L.kl_status(workspace.data_ptr(), _stream(workspace.device))
+
+
+class _FusedKL(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W, kw):
+        out = kl_fwd(H, W, want_row_loss=False, **kw)
+        ctx.save_for_backward(H, W, out["lse_s"], out["lse_t"] if out["lse_t"] is not None
+                              else out["lse_s"])
+        ctx.kw = kw
+        ctx.hidden = out["lse_t"] is not None
+        return out["loss"]
+
+    @staticmethod
+    def backward(ctx, g):
+        H, W, lse_s, lse_t = ctx.saved_tensors
+        out = kl_bwd(H, W, lse_s, lse_t if ctx.hidden else None, grad_loss=g.reshape(()),
+                     **ctx.kw)
+        return out["dH"], out["dW"].to(W.dtype), None
+
+
+def fused_kl_loss(H, W, **kw):
+    """Differentiable loss (w.r.t. H and W) via kl_fwd / kl_bwd."""
+    return _FusedKL.apply(H, W, kw)

@@ -1,0 +1,175 @@
+/*
+ * chunked_kl.h -- C ABI of the fused, chunked distillation KL loss over the
+ * LM output head, for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute ("Efficient Knowledge Distillation for LLMs: Offline
+ * Top-K Logits and a Fused Chunked KL Loss", §1 and §3; KDFlow abstract for the
+ * teacher-hidden mode).  With s = H . W^T the student logits, s~ = s / T,
+ * lse_s = log sum_j exp(s~_j), p_s = softmax(s~):
+ *
+ *   KL_TEACHER_TOPK, partial mass (teacher_lse != NULL; §3 "Offline
+ *   distillation": the cached top-K keeps its unnormalised partial mass):
+ *       q_i = exp(t_i / T - lse_t),  m = sum_i q_i,
+ *       l_n = sum_{i in S_n} q_i (log q_i - s~_{idx_i} + lse_s)
+ *           = [sum q log q] - [sum q_i s~_{idx_i}] + m * lse_s
+ *       (teacher-entropy, cross and mass terms; only lse_s needs the full
+ *       vocabulary).   dl_n/ds_j = (m p_s,j - q_j [j in S_n]) / T.
+ *   KL_TEACHER_TOPK, renormalised (teacher_lse == NULL): q = softmax over the
+ *       row's valid cached entries of t / T, m = 1, same formulas.
+ *   KL_TEACHER_HIDDEN (KDFlow abstract: teacher logits recomputed from the
+ *       teacher's final hidden states through a frozen teacher head):
+ *       t = Ht . Wt^T,  l_n = KL(p_t || p_s),  dl_n/ds_j = (p_s,j - p_t,j) / T.
+ *   loss = (1 / n) sum_{mask_n = 1} l_n, n = normalizer if > 0, else the number
+ *       of rows with mask = 1 (0 valid rows -> loss 0, gradients 0).
+ *   dS = g * dloss/ds (0 on masked rows), dH = dS . W, dW = dS^T . H.
+ *   The teacher head is frozen: no gradient for Ht, Wt.
+ *
+ * The N x V logit tensor is never materialised (§3 "Fused chunked KL"): tokens
+ * are processed in chunks of chunk_tokens rows, and the workspace holds one
+ * chunk's logits, so extra memory is O(chunk_tokens * V + N).
+ *
+ * Conventions for every call below.
+ *   - Every array argument is a DEVICE pointer owned by the caller, except
+ *     kl_problem itself (host memory, read during the call only).
+ *   - Row-major layouts.  H [N, d], W [V, d], Ht [N, d_t], Wt [V, d_t],
+ *     topk_idx/topk_logit [N, K], mask/teacher_lse/lse/row_loss [N],
+ *     dH [N, d] (same dtype as H), dW [V, d] float32.
+ *   - Alignment: H, W, Ht, Wt, dH, dW and the workspace must be 16-byte
+ *     aligned, and d, d_t must make rows a multiple of 16 bytes
+ *     (multiple of 8 for bf16, of 4 for fp32).  Violations return KL_ERR_ALIGN.
+ *   - stream is a cudaStream_t (passed as void*; NULL = legacy default
+ *     stream).  Calls are asynchronous on it; no host synchronisation happens
+ *     inside a call.  Host-detectable errors (NULL, shape, dtype, alignment,
+ *     workspace size, no sm_100 device, launch failure) are returned at once
+ *     and nothing is launched (or nothing further, for a launch failure).
+ *   - Device-detected errors (cache index out of range or duplicated, a
+ *     bounded wait that ran out) are recorded in a status word inside the
+ *     workspace; read it with kl_status().  The kernels stay in bounds and
+ *     finish after such an error, but the outputs are then unspecified.
+ *   - The workspace must be at least kl_workspace_bytes() bytes for the same
+ *     problem and entry point; its contents need not be initialised and are
+ *     not meaningful between calls (except the status word).
+ *   - Not re-entrant on one workspace: calls that share a workspace must be
+ *     ordered (e.g. on one stream).
+ */
+#ifndef CHUNKED_KL_H
+#define CHUNKED_KL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types of H, W, Ht, Wt, dH */
+#define KL_DTYPE_BF16 0 /* bfloat16, tensor-core kind::f16, fp32 accumulation */
+#define KL_DTYPE_F32 1  /* float32, tensor-core kind::tf32, fp32 accumulation  */
+
+/* teacher modes */
+#define KL_TEACHER_TOPK 0   /* offline cache: topk_idx, topk_logit (+ teacher_lse) */
+#define KL_TEACHER_HIDDEN 1 /* teacher hidden states Ht through frozen head Wt     */
+
+/* entry points, for kl_workspace_bytes */
+#define KL_ENTRY_FWD 0
+#define KL_ENTRY_BWD 1
+#define KL_ENTRY_FWD_BWD 2
+
+/* status codes (return values of the calls and of kl_status) */
+#define KL_OK 0
+#define KL_ERR_NULL 1        /* a required pointer is NULL                         */
+#define KL_ERR_SHAPE 2       /* a size is out of range (N<0, d<1, V<1, K<1, ...)     */
+#define KL_ERR_DTYPE 3       /* unknown dtype or teacher mode                      */
+#define KL_ERR_ALIGN 4       /* pointer or row stride not 16-byte aligned          */
+#define KL_ERR_WORKSPACE 5   /* ws_bytes < kl_workspace_bytes()                    */
+#define KL_ERR_CUDA 6        /* a CUDA runtime call or kernel launch failed        */
+#define KL_ERR_INDEX 7       /* device: cache index outside [-1, V) or duplicated  */
+#define KL_ERR_TIMEOUT 8     /* device: a bounded wait inside a kernel ran out     */
+#define KL_ERR_UNSUPPORTED 9 /* the current device is not sm_100 (B200-class)      */
+#define KL_ERR_ARG 10        /* another bad argument (T <= 0, chunk_tokens < 0...) */
+
+typedef struct kl_problem {
+  int64_t N;           /* tokens (rows of H); N = 0 gives loss 0 and no gradient */
+  int64_t d;           /* student hidden width                                  */
+  int64_t V;           /* vocabulary size (rows of W)                           */
+  int32_t dtype;       /* KL_DTYPE_*: element type of H, W, Ht, Wt and dH       */
+  int32_t teacher;     /* KL_TEACHER_*                                          */
+  const void* H;       /* [N, d] student hidden states                          */
+  const void* W;       /* [V, d] student output head (nn.Linear layout)         */
+  const uint8_t* mask; /* [N] 1 = keep, 0 = ignore; NULL = keep all             */
+  float T;             /* temperature, > 0, divides student and teacher logits  */
+  int32_t K;           /* TOPK: cached entries per row, 1..1024                  */
+  const int32_t* topk_idx;   /* TOPK: [N, K] vocabulary ids; -1 = empty slot     */
+  const float* topk_logit;   /* TOPK: [N, K] teacher logits t (before / T)       */
+  const float* teacher_lse;  /* TOPK: [N] log sum_j exp(t_j / T) over the full
+                                vocabulary (partial mass), or NULL (renormalise) */
+  int64_t d_t;               /* HIDDEN: teacher hidden width                     */
+  const void* Ht;            /* HIDDEN: [N, d_t] teacher final hidden states     */
+  const void* Wt;            /* HIDDEN: [V, d_t] frozen teacher output head      */
+  int64_t chunk_tokens;      /* token rows per chunk; 0 = library default (4096) */
+  float normalizer;          /* > 0: divide by this (e.g. a data-parallel global
+                                count) instead of the number of unmasked rows    */
+} kl_problem;
+
+/* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if
+ * the problem is invalid.  O(chunk_tokens * V + N * 16), never O(N * V). */
+size_t kl_workspace_bytes(const kl_problem* p, int entry);
+
+/* Forward only.  Writes loss (device float scalar), lse_s [N] (log-sum-exp of
+ * s~ per row, needed by kl_bwd), lse_t [N] (HIDDEN: teacher log-sum-exp; may be
+ * NULL in TOPK mode) and row_loss [N] (per-row l_n, 0 on masked rows; may be
+ * NULL).  Tensor work: 2 N d V (+ 2 N d_t V in HIDDEN mode). */
+int kl_fwd(const kl_problem* p, void* ws, size_t ws_bytes, float* loss, float* lse_s,
+           float* lse_t, float* row_loss, void* stream);
+
+/* Backward, recomputing each chunk's logits from H and W (output-head gradient
+ * checkpointing, §3 "Fused chunked KL").  lse_s (and lse_t in HIDDEN mode) come
+ * from kl_fwd on the same inputs.  grad_loss is a DEVICE pointer to the
+ * incoming scalar gradient g.  Writes dH [N, d]; writes dW [V, d] fp32, or adds
+ * to it when accumulate_dW != 0.  Tensor work: 6 N d V (+ 2 N d_t V). */
+int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,
+           const float* lse_t, const float* grad_loss, void* dH, float* dW,
+           int accumulate_dW, void* stream);
+
+/* Fused forward + backward in one pass over the chunks (the logits of a chunk
+ * are computed once and turned into dS in place).  grad_loss is the incoming
+ * scalar gradient g by value.  Writes loss (device scalar), row_loss [N] (may
+ * be NULL), dH, and dW (overwrite, or accumulate if accumulate_dW != 0).
+ * Tensor work: 6 N d V (+ 2 N d_t V in HIDDEN mode). */
+int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss,
+               float* loss, float* row_loss, void* dH, float* dW, int accumulate_dW,
+               void* stream);
+
+/* Synchronises stream, then returns the device-side status recorded in ws
+ * (KL_OK, KL_ERR_INDEX or KL_ERR_TIMEOUT), or KL_ERR_CUDA if the stream
+ * reports an error.  Does not clear it; every kl_* call resets it at start. */
+int kl_status(void* ws, void* stream);
+
+/* Static English description of a status code. */
+const char* kl_status_string(int code);
+
+/* Kernel launches issued by this library since it was loaded. */
+uint64_t kl_launch_count(void);
+
+/* Per-kernel timing with CUDA events recorded on the launch stream around each
+ * launch.  kl_profile_begin() clears and enables it; kl_profile_end()
+ * synchronises the recorded events, disables recording and fills up to
+ * max_entries entries (one per kernel kind that launched); returns the number
+ * of kinds, or -KL_ERR_CUDA.  flops is the algorithmic work of all launches
+ * of that kind (2 M N K for the tensor-core contractions, 0 otherwise);
+ * bytes is the algorithmic HBM traffic of the memory-bound kernels. */
+typedef struct kl_profile_entry {
+  char name[48];
+  uint64_t launches;
+  double total_ms;
+  double flops;
+  double bytes;
+} kl_profile_entry;
+int kl_profile_begin(void);
+int kl_profile_end(kl_profile_entry* out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CHUNKED_KL_H */

@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, sizes workspaces as O(chunk * V + N), and rejects bad
+arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunked_kl_loss_tma_b200 import _lib as L
+from chunked_kl_loss_tma_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "chunked_kl.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_\s\*]*?\b(kl_[a-z_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_functions():
+    assert _declared() == sorted(L.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def _problem(**kw):
+    p = L.KLProblem()
+    p.N, p.d, p.V, p.dtype, p.teacher, p.K, p.T = 4096, 3072, 128256, 0, 0, 64, 1.0
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_workspace_is_chunk_sized_not_NV(lib):
+    small = L.kl_workspace_bytes(_problem(N=4096), L.KL_ENTRY_FWD_BWD)
+    big = L.kl_workspace_bytes(_problem(N=262144), L.KL_ENTRY_FWD_BWD)
+    # one [4096, V] bf16 logit chunk + per-chunk stats; growth with N is O(N) only
+    assert small >= 4096 * 128256 * 2
+    assert big - small <= (262144 - 4096) * 8 + 4096
+    assert big < 262144 * 128256 * 2 / 10
+    assert L.kl_workspace_bytes(_problem(chunk_tokens=1024), 2) < small
+
+
+def test_workspace_hidden_mode_has_two_logit_buffers(lib):
+    p = _problem(teacher=1, d_t=4096, K=0)
+    assert L.kl_workspace_bytes(p, 2) >= 2 * 4096 * 128256 * 2
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d", 3070, 4),           # rows not 16-byte aligned -> KL_ERR_ALIGN
+    ("dtype", 7, 3),          # KL_ERR_DTYPE
+    ("teacher", 5, 3),
+    ("K", 0, 2),              # KL_ERR_SHAPE
+    ("K", 1025, 2),
+    ("V", 0, 2),
+    ("N", -1, 2),
+    ("T", 0.0, 10),           # KL_ERR_ARG
+    ("T", -1.0, 10),
+    ("chunk_tokens", -5, 10),
+])
+def test_bad_problems_rejected_on_host(lib, field, value, code):
+    p = _problem(**{field: value})
+    assert L.kl_workspace_bytes(p, 2) == 0
+    p.H = p.W = p.topk_idx = p.topk_logit = 256
+    rc = L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None)
+    assert rc == code, (rc, L.kl_status_string(rc))
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _problem()
+    assert L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None) == 1
+    p.H, p.W, p.topk_idx, p.topk_logit = 264, 256, 256, 256
+    assert L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None) == 4
+    p.H = 272
+    # valid arguments: without a CUDA device the call fails with KL_ERR_CUDA
+    import torch
+    if not torch.cuda.is_available():
+        assert L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None) == 6
+
+
+def test_status_strings(lib):
+    for code, name in L.STATUS.items():
+        assert L.kl_status_string(code) and isinstance(L.kl_status_string(code), str)
+    assert lib.kl_launch_count() >= 0

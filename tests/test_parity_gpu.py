@@ -1,0 +1,224 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerances (stated by the loss's accuracy target): loss relative error
+<= 1e-3; dH and dW max-abs error <= 2e-2 * max|oracle gradient| for bf16 inputs
+with fp32 accumulation (and for fp32 inputs through tf32 tensor cores).
+Shapes are chosen to span several 128 x 256 tiles with ragged tails in every
+dimension (N, d, V not tile multiples, several token chunks with a short
+last one)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_tma_b200 import _lib as L
+from chunked_kl_loss_tma_b200 import ops
+from chunked_kl_loss_tma_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-3
+GRAD_FRAC = 2e-2
+
+
+def _oracle(w, **kw):
+    args = dict(T=w.T, mask=w.mask, mode=w.mode)
+    if w.mode == "topk":
+        args.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        args.update(Ht=w.Ht, Wt=w.Wt)
+    args.update(kw)
+    return oracle.kl_loss(w.H, w.W, **args)
+
+
+def _kw(w, chunk=0, normalizer=0.0):
+    kw = dict(T=w.T, mask=w.mask, chunk_tokens=chunk, normalizer=normalizer)
+    if w.mode == "topk":
+        kw.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        kw.update(Ht=w.Ht, Wt=w.Wt)
+    return kw
+
+
+def _check_grad(got, ref, name):
+    got = got.detach().double().cpu().numpy()
+    scale = np.max(np.abs(ref))
+    err = np.max(np.abs(got - ref))
+    assert err <= GRAD_FRAC * scale, f"{name}: max abs err {err:.3e} > {GRAD_FRAC} * {scale:.3e}"
+    return err / scale
+
+
+def _check_loss(got, ref):
+    got = float(got)
+    assert abs(got - ref) <= LOSS_RTOL * max(abs(ref), 1e-30), f"loss {got} vs oracle {ref}"
+
+
+def _small_topk(N=300, d=200, V=5003, K=16, dtype=torch.bfloat16, T=1.3, seed=11,
+                partial=True, masked=True):
+    w = wl.make_topk("small_topk", N=N, d=d, V=V, K=K, d_t=64, T=T, dtype=dtype,
+                     w_std=0.05, tw_std=0.1, seed=seed, partial_mass=partial)
+    if masked:
+        m = torch.ones(N, dtype=torch.uint8)
+        m[::7] = 0
+        w.mask = m
+    return w.to("cuda")
+
+
+def _small_hidden(N=200, d=136, d_t=72, V=3001, dtype=torch.bfloat16, T=2.0, seed=12):
+    w = wl.make_hidden("small_hidden", N=N, d=d, d_t=d_t, V=V, T=T, dtype=dtype,
+                       w_std=0.08, tw_std=0.1, seed=seed)
+    m = torch.ones(N, dtype=torch.uint8)
+    m[3::5] = 0
+    w.mask = m
+    return w.to("cuda")
+
+
+@pytest.mark.parametrize("partial", [True, False])
+def test_tiny_fp32_fwd_bwd(partial):
+    w = wl.tiny(partial_mass=partial).to("cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w))
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(out["row_loss"].cpu().numpy(), ref["row_loss"], rtol=2e-3,
+                               atol=1e-5)
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    assert ops.status(out["workspace"]) == 0
+
+
+@pytest.mark.parametrize("partial", [True, False])
+@pytest.mark.parametrize("chunk", [128, 0])
+def test_bf16_topk_ragged_fwd_bwd(partial, chunk):
+    w = _small_topk(partial=partial)
+    out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=1.7, want_row_loss=True, **_kw(w, chunk))
+    ref = _oracle(w, grad_loss=1.7)
+    _check_loss(out["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(out["row_loss"].cpu().numpy(), ref["row_loss"], rtol=5e-3,
+                               atol=2e-4)
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    assert ops.status(out["workspace"]) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_hidden_mode_fwd_bwd(dtype):
+    w = _small_hidden(dtype=dtype)
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w, chunk=96))
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(out["row_loss"].cpu().numpy(), ref["row_loss"], rtol=5e-3,
+                               atol=2e-4)
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+@pytest.mark.parametrize("mode", ["topk", "hidden"])
+def test_split_fwd_then_bwd(mode):
+    w = _small_topk() if mode == "topk" else _small_hidden()
+    kw = _kw(w, chunk=128)
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    ref = _oracle(w, grad_loss=0.6)
+    _check_loss(f["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(f["lse_s"].cpu().numpy(), ref["lse_s"], rtol=1e-5, atol=1e-5)
+    if mode == "hidden":
+        np.testing.assert_allclose(f["lse_t"].cpu().numpy(), ref["lse_t"], rtol=1e-5, atol=1e-5)
+    g = torch.full((), 0.6, device="cuda")
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"], grad_loss=g, **kw)
+    _check_grad(b["dH"], ref["dH"], "dH")
+    _check_grad(b["dW"], ref["dW"], "dW")
+
+
+def test_autograd_function_matches_oracle():
+    w = _small_topk(N=160, V=2100, masked=False)
+    H = w.H.clone().requires_grad_(True)
+    W = w.W.clone().requires_grad_(True)
+    kw = _kw(w)
+    loss = ops.fused_kl_loss(H, W, **kw)
+    (2.0 * loss).backward()
+    ref = _oracle(w, grad_loss=2.0)
+    _check_loss(loss.item(), ref["loss"])
+    _check_grad(H.grad, ref["dH"], "dH")
+    _check_grad(W.grad.float(), ref["dW"], "dW")
+
+
+def test_accumulate_dW_and_chunk_invariance():
+    w = _small_topk(seed=21)
+    kw = _kw(w, chunk=64)
+    base = torch.randn(w.W.shape, device="cuda", dtype=torch.float32)
+    dW = base.clone()
+    out = ops.kl_fwd_bwd(w.H, w.W, dW=dW, accumulate_dW=True, **kw)
+    ref = _oracle(w)
+    _check_grad(out["dW"] - base, ref["dW"], "accumulated dW")
+    other = ops.kl_fwd_bwd(w.H, w.W, **_kw(w, chunk=1000))
+    assert abs(out["loss"].item() - other["loss"].item()) <= 1e-5 * abs(other["loss"].item())
+    _check_grad(other["dH"], out["dH"].double().cpu().numpy(), "dH across chunk sizes")
+
+
+def test_normalizer_override():
+    w = _small_topk(seed=22)
+    out = ops.kl_fwd_bwd(w.H, w.W, **_kw(w, normalizer=1000.0))
+    ref = _oracle(w, normalizer=1000.0)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_topk_K_equals_V_matches_full_kl():
+    V, N = 320, 96
+    w = wl.make_topk("kv", N=N, d=64, V=V, K=V, d_t=32, T=1.0, dtype=torch.bfloat16,
+                     w_std=0.1, tw_std=0.2, seed=23).to("cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, **_kw(w))
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_empty_slots_and_all_masked_rows():
+    w = _small_topk(seed=24, masked=False)
+    idx = w.topk_idx.clone()
+    idx[:, -3:] = -1
+    idx[5, :] = -1  # a row with no cached entry contributes 0
+    w.topk_idx = idx
+    out = ops.kl_fwd_bwd(w.H, w.W, **_kw(w))
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dW"], ref["dW"], "dW")
+    w.mask = torch.zeros(w.N, dtype=torch.uint8, device="cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, **_kw(w))
+    assert out["loss"].item() == 0.0
+    assert out["dH"].abs().max().item() == 0.0 and out["dW"].abs().max().item() == 0.0
+
+
+def test_empty_problem():
+    H = torch.empty(0, 64, device="cuda", dtype=torch.bfloat16)
+    W = torch.randn(100, 64, device="cuda").to(torch.bfloat16)
+    idx = torch.empty(0, 4, dtype=torch.int32, device="cuda")
+    val = torch.empty(0, 4, dtype=torch.float32, device="cuda")
+    out = ops.kl_fwd_bwd(H, W, topk_idx=idx, topk_logit=val)
+    assert out["loss"].item() == 0.0 and out["dW"].abs().max().item() == 0.0
+
+
+def test_bad_cache_index_sets_device_status():
+    w = _small_topk(seed=25)
+    idx = w.topk_idx.clone()
+    idx[7, 2] = w.V + 5
+    out = ops.kl_fwd_bwd(w.H, w.W, **dict(_kw(w), topk_idx=idx))
+    assert ops.status(out["workspace"]) == 7  # KL_ERR_INDEX
+    idx = w.topk_idx.clone()
+    idx[9, 1] = idx[9, 0]
+    out = ops.kl_fwd_bwd(w.H, w.W, **dict(_kw(w), topk_idx=idx))
+    assert ops.status(out["workspace"]) == 7
+    ok = ops.kl_fwd_bwd(w.H, w.W, **_kw(w))  # status resets on the next call
+    assert ops.status(ok["workspace"]) == 0
+
+
+def test_launch_counter_and_profile():
+    w = _small_topk(seed=26)
+    before = L.kl_launch_count()
+    L.kl_profile_begin()
+    ops.kl_fwd_bwd(w.H, w.W, **_kw(w, chunk=128))
+    prof = L.kl_profile_end()
+    names = {p["name"] for p in prof}
+    assert {"gemm_logits_stats", "gemm_dH", "gemm_dW", "dlogits_topk"} <= names
+    assert L.kl_launch_count() - before == sum(p["launches"] for p in prof)
+    assert all(p["total_ms"] > 0 for p in prof)
