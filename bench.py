@@ -25,7 +25,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -122,9 +121,9 @@ def gpu_arm(args):
     import torch
     import torch.distributed as dist
 
-    import chunked_kl_loss_tma_b200 as ckl
     from chunked_kl_loss_tma_b200 import _lib, ops
     from chunked_kl_loss_tma_b200 import workloads as wl
+    from chunked_kl_loss_tma_b200.dist import max_over_ranks
 
     ws, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
@@ -180,10 +179,8 @@ def gpu_arm(args):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     peak_extra = torch.cuda.max_memory_allocated(dev) - base_mem
-    elapsed = torch.tensor([ms], dtype=torch.float64, device=dev)
     if ws > 1:
-        dist.all_reduce(elapsed, op=dist.ReduceOp.MAX)
-    ms = float(elapsed.item())
+        ms = max_over_ranks(ms)
 
     # ---- end to end through the public API: pinned host inputs in, loss out
     e2e = None
@@ -216,11 +213,11 @@ def gpu_arm(args):
             e2e_step()
         e1.record()
         barrier()
-        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        ems = e0.elapsed_time(e1)
         if ws > 1:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+            ems = max_over_ranks(ems)
         h2d = sum(t.numel() * t.element_size() for t in (hH, hidx, hval, hlse))
-        e2e = {"value": ws * args.N * args.steps / (float(ems.item()) / 1e3),
+        e2e = {"value": ws * args.N * args.steps / (ems / 1e3),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
 
     if ws > 1:
