@@ -21,12 +21,14 @@ KL_ENTRY_FWD_BWD = 2
 STATUS = {
     0: "KL_OK", 1: "KL_ERR_NULL", 2: "KL_ERR_SHAPE", 3: "KL_ERR_DTYPE", 4: "KL_ERR_ALIGN",
     5: "KL_ERR_WORKSPACE", 6: "KL_ERR_CUDA", 7: "KL_ERR_INDEX", 8: "KL_ERR_TIMEOUT",
-    9: "KL_ERR_UNSUPPORTED", 10: "KL_ERR_ARG",
+    9: "KL_ERR_UNSUPPORTED", 10: "KL_ERR_ARG", 11: "KL_ERR_TOO_LARGE",
 }
+KL_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol declared in include/chunked_kl.h.
 EXPORTS = ("kl_workspace_bytes", "kl_fwd", "kl_bwd", "kl_fwd_bwd", "kl_status",
-           "kl_status_string", "kl_launch_count", "kl_profile_begin", "kl_profile_end")
+           "kl_status_string", "kl_launch_count", "kl_profile_begin", "kl_profile_end",
+           "kl_fwd_noalloc")
 
 
 class KLProblem(ctypes.Structure):
@@ -76,6 +78,8 @@ def lib():
     L.kl_bwd.restype = i32
     L.kl_fwd_bwd.argtypes = [P, vp, sz, f32, vp, vp, vp, vp, i32, vp]
     L.kl_fwd_bwd.restype = i32
+    L.kl_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
+    L.kl_fwd_noalloc.restype = i32
     L.kl_status.argtypes = [vp, vp]
     L.kl_status.restype = i32
     L.kl_status_string.argtypes = [i32]
@@ -118,6 +122,12 @@ def kl_bwd(prob, ws, ws_bytes, lse_s, lse_t, grad_loss, dH, dW, accumulate_dW, s
 def kl_fwd_bwd(prob, ws, ws_bytes, grad_loss, loss, row_loss, dH, dW, accumulate_dW, stream):
     return lib().kl_fwd_bwd(ctypes.byref(prob), ws, ws_bytes, float(grad_loss), loss, row_loss,
                             dH, dW, int(accumulate_dW), stream)
+
+
+def kl_fwd_noalloc(prob, loss, lse_s, row_loss, status, stream):
+    """Forward with the library's fixed static scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/chunked_kl.h)."""
+    return lib().kl_fwd_noalloc(ctypes.byref(prob), loss, lse_s, row_loss, status, stream)
 
 
 def kl_status(ws, stream):

@@ -782,6 +782,8 @@ const char* kl_status_string(int code) {
     case KL_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case KL_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200-class)";
     case KL_ERR_ARG: return "bad argument (temperature, chunk size or normaliser)";
+    case KL_ERR_TOO_LARGE:
+      return "problem needs more scratch than kl_fwd_noalloc's fixed array holds";
     default: return "unknown status";
   }
 }
@@ -828,3 +830,84 @@ int kl_profile_end(kl_profile_entry* out, int max_entries) {
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation forward
+// Scratch for kl_fwd_noalloc: one fixed array in static device memory, so the
+// call needs neither cudaMalloc nor a caller workspace.  Host code only names
+// it through the address looked up below (the host-side symbol is a stand-in,
+// not a device address).
+static __device__ __align__(256) uint8_t g_noalloc_scratch[KL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+uint8_t* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current.
+int noalloc_scratch(uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return KL_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<uint8_t*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return KL_OK;
+}
+}  // namespace
+
+extern "C" int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
+                              int* status, void* stream) {
+  KL_TRY(validate(p));
+  if (p->dtype != KL_DTYPE_BF16 || p->teacher != KL_TEACHER_TOPK) return KL_ERR_DTYPE;
+  if (loss == nullptr || (p->N > 0 && (lse_s == nullptr || row_loss == nullptr)))
+    return KL_ERR_NULL;
+  DevInfo di;
+  KL_TRY(current_device_info(&di));
+  // Layout in the fixed array: scalars | tile statistics | sorted ids | q | (m, sum q log q).
+  const int64_t tiles_v = cdiv(p->V, kBN);
+  const size_t per_row = static_cast<size_t>(tiles_v) * sizeof(float4) +
+                         static_cast<size_t>(p->K) * 8 + sizeof(float2);
+  const size_t fixed = 256 + 4 * 256;  // header + alignment of the four regions
+  if (per_row + fixed > KL_NOALLOC_SCRATCH_BYTES) return KL_ERR_TOO_LARGE;
+  int64_t C = static_cast<int64_t>((KL_NOALLOC_SCRATCH_BYTES - fixed) / per_row);
+  if (p->chunk_tokens > 0 && p->chunk_tokens < C) C = p->chunk_tokens;
+  if (p->N < C) C = p->N > 0 ? p->N : 1;
+  uint8_t* scratch = nullptr;
+  KL_TRY(noalloc_scratch(&scratch));
+  Ctx c;
+  c.p = p;
+  c.pl.eb = 2;
+  c.pl.C = C;
+  c.pl.Vp = cdiv(p->V, 8) * 8;
+  c.pl.tiles_v = static_cast<int>(tiles_v);
+  c.pl.hidden = false;
+  size_t off = 256;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  c.pl.off_ps = take(static_cast<size_t>(C) * tiles_v * sizeof(float4));
+  c.pl.off_sidx = take(static_cast<size_t>(C) * p->K * 4);
+  c.pl.off_sq = take(static_cast<size_t>(C) * p->K * 4);
+  c.pl.off_rinfo = take(static_cast<size_t>(C) * sizeof(float2));
+  c.pl.total = off;
+  if (c.pl.total > KL_NOALLOC_SCRATCH_BYTES) return KL_ERR_TOO_LARGE;
+  c.ws = scratch;
+  c.sc = reinterpret_cast<Scalars*>(scratch);
+  c.st = static_cast<cudaStream_t>(stream);
+  c.sms = di.sms;
+  c.invT = 1.0f / p->T;
+  // run_fwd resets the status word first and overwrites every scratch region
+  // before reading it, so the previous call's contents do not leak in.
+  KL_TRY(run_fwd<__nv_bfloat16>(c, loss, lse_s, nullptr, row_loss));
+  if (status != nullptr &&
+      cudaMemcpyAsync(status, &c.sc->status, sizeof(int), cudaMemcpyDeviceToDevice, c.st) !=
+          cudaSuccess)
+    return KL_ERR_CUDA;
+  return KL_OK;
+}

@@ -87,6 +87,8 @@ extern "C" {
 #define KL_ERR_TIMEOUT 8     /* device: a bounded wait inside a kernel ran out     */
 #define KL_ERR_UNSUPPORTED 9 /* the current device is not sm_100 (B200-class)      */
 #define KL_ERR_ARG 10        /* another bad argument (T <= 0, chunk_tokens < 0...) */
+#define KL_ERR_TOO_LARGE 11  /* kl_fwd_noalloc: one token row needs more than the
+                                fixed KL_NOALLOC_SCRATCH_BYTES of scratch          */
 
 typedef struct kl_problem {
   int64_t N;           /* tokens (rows of H); N = 0 gives loss 0 and no gradient */
@@ -139,6 +141,37 @@ int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,
 int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss,
                float* loss, float* row_loss, void* dH, float* dW, int accumulate_dW,
                void* stream);
+
+/* Forward-only variant for callers that cannot allocate device memory.
+ *
+ * No counterpart in the paper: this is a deployment convenience.  Some callers
+ * cannot call cudaMalloc or hand over a workspace -- for example a plugin host
+ * that passes only its input and output buffers, a runtime whose device memory
+ * is planned up front and may not grow, or a code path where an allocation
+ * would synchronise the device.  kl_fwd_noalloc computes what kl_fwd computes
+ * (top-K mode, bf16 inputs only) without allocating anything and without a
+ * workspace argument: its scratch (per-chunk tile statistics and the prepared
+ * cache) lives in one fixed array of KL_NOALLOC_SCRATCH_BYTES in the library's
+ * static device memory, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ * Arguments: as kl_fwd, except that row_loss [N] is required, lse_t is not
+ * used, and status (device int, may be NULL) receives the device-side status
+ * (KL_OK / KL_ERR_INDEX / KL_ERR_TIMEOUT) once the call's kernels finish.
+ * The token chunk is the largest that fits the fixed scratch (and at most
+ * chunk_tokens when that is set); results match kl_fwd up to rounding order.
+ * Errors: KL_ERR_DTYPE unless bf16 + KL_TEACHER_TOPK; KL_ERR_TOO_LARGE when a
+ * single token row of scratch (16 * ceil(V / 256) + 8 * K + 8 bytes, plus a
+ * 256-byte header) exceeds KL_NOALLOC_SCRATCH_BYTES; the other codes as kl_fwd.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.  The first call
+ * on a device looks up the scratch array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents (each
+ * call re-initialises what it reads), so calls whose kernels overlap on the GPU
+ * (different streams, or different host threads) race: order them. */
+#define KL_NOALLOC_SCRATCH_BYTES (16u << 20)
+int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
+                   int* status, void* stream);
 
 /* Synchronises stream, then returns the device-side status recorded in ws
  * (KL_OK, KL_ERR_INDEX or KL_ERR_TIMEOUT), or KL_ERR_CUDA if the stream
