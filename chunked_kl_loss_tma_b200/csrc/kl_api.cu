@@ -190,10 +190,36 @@ struct Plan {
   // current chunk of H or Ht) and K-major copies W^T [d][Vp], dS^T [V][Cp],
   // H_c^T [d][Cp] for the gradient contractions.
   int64_t Cp = 0;
+  int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
+  size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
   size_t off_wr = 0, off_wtr = 0, off_xr = 0, off_wT = 0, off_sT = 0, off_hT = 0;
 };
 
 // Sizes, dtypes and scalar arguments (no pointers).
+// Number of K-parts for a contraction with `tiles` output tiles and `num_kb`
+// K-blocks on `units` CTA pairs: the smallest split (at most 8, each part at
+// least 32 K-blocks) whose last wave is fullest.  Every part is non-empty.
+int choose_ksplit(int64_t tiles, int64_t num_kb, int64_t units) {
+  int best = 1;
+  double best_eff = 0;
+  for (int s = 1; s <= 8; ++s) {
+    if (num_kb / s < 32 && s > 1) break;
+    const int64_t kbs = cdiv(num_kb, s);
+    if ((s - 1) * kbs >= num_kb) continue;  // an empty part
+    const int64_t u = tiles * s;
+    const double eff = static_cast<double>(u) / (cdiv(u, units) * units);
+    if (eff > best_eff + 0.01) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// CTA pairs available for one contraction (the workspace plan must not depend
+// on the device, so this is the B200's 148 SMs / 2).
+int64_t max_units_hint() { return 74; }
+
 int validate_shape(const kl_problem* p) {
   if (p == nullptr) return KL_ERR_NULL;
   if (p->dtype != KL_DTYPE_BF16 && p->dtype != KL_DTYPE_F32) return KL_ERR_DTYPE;
@@ -264,6 +290,12 @@ Plan make_plan(const kl_problem* p, int entry) {
     if (pl.hidden) pl.off_lse_t = take(nrow);
   }
   if (entry != KL_ENTRY_BWD) pl.off_rl = take(nrow);
+  if (pl.eb == 2 && entry != KL_ENTRY_FWD) {
+    pl.ksplit_dh = choose_ksplit(cdiv(pl.C, 2 * kBM) * cdiv(p->d, kBN), cdiv(p->V, 64),
+                                 max_units_hint());
+    if (pl.ksplit_dh > 1)
+      pl.off_dhp = take(static_cast<size_t>(pl.ksplit_dh) * pl.C * p->d * 4);
+  }
   if (pl.eb == 4) {
     const int64_t dmax = (pl.hidden && p->d_t > p->d) ? p->d_t : p->d;
     pl.off_wr = take(static_cast<size_t>(p->V) * p->d * 4);
@@ -281,10 +313,10 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, GemmParams gp, double flops) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI>;
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -295,12 +327,28 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
     attr_set[dev] = true;
   }
   const int tiles = gp.tiles_m * gp.tiles_n;
-  const int grid = tiles < sms ? tiles : sms;
+  const int units = PAIR ? sms / 2 : sms;  // CTA pairs or CTAs, one CTA per SM
+  const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    kern<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(ma, mb, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, gp);
   }
-  return cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA;
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
 
 #define KL_LAUNCHED() (cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA)
@@ -355,10 +403,10 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
     xc = reinterpret_cast<const uint8_t*>(xr);
   }
   if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
-      !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN))
+      !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2))
     return KL_ERR_CUDA;
   GemmParams gp{};
-  gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+  gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
   gp.tiles_n = c.pl.tiles_v;
   gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
   gp.m_fastest = 1;
@@ -374,8 +422,8 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.ktop = ktop;
   gp.status = &c.sc->status;
   gp.spin_limit = spin_limit();
-  return launch_gemm<Elem, 0, 0, EPI_STATS>(name, c.st, c.sms, ma, mb, gp,
-                                            2.0 * Cn * p->V * dx);
+  return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, gp,
+                                               2.0 * Cn * p->V * dx);
 }
 
 int launch_transpose(Ctx& c, const float* src, int64_t ld_src, float* dst, int64_t ld_dst,
@@ -401,10 +449,10 @@ int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* d
   {
     CUtensorMap ma, mb;
     if (!make_map(&ma, dS, p->dtype, V, Cn, c.pl.Vp * 4, 32, kBM) ||
-        !make_map(&mb, wT, p->dtype, V, d, c.pl.Vp * 4, 32, kBN))
+        !make_map(&mb, wT, p->dtype, V, d, c.pl.Vp * 4, 32, kBN / 2))
       return KL_ERR_CUDA;
     GemmParams gp{};
-    gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+    gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(V, 32));
     gp.m_fastest = 1;
@@ -414,16 +462,16 @@ int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* d
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<float, 0, 0, EPI_STORE>("gemm_dH", c.st, c.sms, ma, mb, gp,
-                                                2.0 * Cn * V * d)));
+    KL_TRY((launch_gemm<float, 0, 0, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+                                                   2.0 * Cn * V * d)));
   }
   {
     CUtensorMap ma, mb;
     if (!make_map(&ma, sT, p->dtype, Cn, V, Cp * 4, 32, kBM) ||
-        !make_map(&mb, hT, p->dtype, Cn, d, Cp * 4, 32, kBN))
+        !make_map(&mb, hT, p->dtype, Cn, d, Cp * 4, 32, kBN / 2))
       return KL_ERR_CUDA;
     GemmParams gp{};
-    gp.tiles_m = static_cast<int>(cdiv(V, kBM));
+    gp.tiles_m = static_cast<int>(cdiv(V, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(Cn, 32));
     gp.m_fastest = 0;
@@ -434,8 +482,8 @@ int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* d
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<float, 0, 0, EPI_ACCUM>("gemm_dW", c.st, c.sms, ma, mb, gp,
-                                                2.0 * Cn * V * d)));
+    KL_TRY((launch_gemm<float, 0, 0, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, gp,
+                                                   2.0 * Cn * V * d)));
   }
   return KL_OK;
 }
@@ -449,25 +497,43 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
   constexpr int kMNe = kRowBytes / sizeof(Elem);
   const int64_t d = p->d;
   const uint64_t ldS = c.pl.Vp * sizeof(Elem);
-  // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.
+  // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.  When the
+  // output has too few tiles to fill the GPU, V is split into ksplit parts whose
+  // fp32 partial products are summed in a fixed order afterwards.
   {
     CUtensorMap ma, mb;
     if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kBKe, kBM) ||
         !make_map(&mb, p->W, p->dtype, d, p->V, d * sizeof(Elem), kMNe, kBKe))
       return KL_ERR_CUDA;
     GemmParams gp{};
-    gp.tiles_m = static_cast<int>(cdiv(Cn, kBM));
+    gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(p->V, kBKe));
     gp.m_fastest = 1;
-    gp.out = static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem);
     gp.ld_out = d;
     gp.rows_valid = static_cast<int>(Cn);
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE>("gemm_dH", c.st, c.sms, ma, mb, gp,
-                                               2.0 * Cn * p->V * d)));
+    int ks = choose_ksplit(static_cast<int64_t>(gp.tiles_m) * gp.tiles_n, gp.num_kb, c.sms / 2);
+    if (ks > c.pl.ksplit_dh) ks = c.pl.ksplit_dh;
+    if (ks > 1) {
+      float* part = reinterpret_cast<float*>(c.ws + c.pl.off_dhp);
+      gp.ksplit = ks;
+      gp.split_stride = Cn * d;
+      gp.out = part;
+      gp.beta = 0;
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+                                                    2.0 * Cn * p->V * d)));
+      LaunchScope ls("splitk_reduce", c.st, 0, (4.0 * ks + sizeof(Elem)) * Cn * d);
+      splitk_reduce_kernel<Elem><<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(
+          part, ks, Cn * d, static_cast<Elem*>(dH) + c0 * d, Cn * d);
+      KL_TRY(cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA);
+    } else {
+      gp.out = static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem);
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+                                                    2.0 * Cn * p->V * d)));
+    }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
   {
@@ -477,7 +543,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
         !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe))
       return KL_ERR_CUDA;
     GemmParams gp{};
-    gp.tiles_m = static_cast<int>(cdiv(p->V, kBM));
+    gp.tiles_m = static_cast<int>(cdiv(p->V, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(Cn, kBKe));
     gp.m_fastest = 0;
@@ -488,8 +554,8 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM>("gemm_dW", c.st, c.sms, ma, mb, gp,
-                                               2.0 * Cn * p->V * d)));
+    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, gp,
+                                                  2.0 * Cn * p->V * d)));
   }
   return KL_OK;
 }

@@ -15,6 +15,15 @@
 //   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
 //   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, read-modify-write across chunks.
 //
+// Two tile shapes: PAIR = 0, one CTA computes a 128 x 256 tile with
+// tcgen05.mma.cta_group::1; PAIR = 1, a cluster of two CTAs (one per SM)
+// computes a 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA loads its
+// own 128 rows of A and its own 128-row half of B, only the leader CTA issues
+// the MMAs, both CTAs' loads complete on the leader's barriers, the leader's
+// commits arrive on both CTAs' barriers, and each CTA's epilogue reads its own
+// 128 accumulator rows from its own TMEM.  The pair halves the operand bytes
+// each SM stages per MMA.
+//
 // Roles (192 threads, one CTA per SM, grid-strided over output tiles):
 //   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
@@ -36,7 +45,8 @@ namespace ckl {
 
 constexpr int kBM = 128;          // tile rows (TMEM lanes)
 constexpr int kBN = 256;          // tile columns (TMEM columns per accumulator)
-constexpr int kStages = 4;        // smem ring depth
+constexpr int kStages = 4;        // smem ring depth (1-CTA tiles)
+constexpr int kStagesPair = 6;    // smem ring depth (2-CTA tiles: 32 KB stages)
 constexpr int kRowBytes = 128;    // one 128-B swizzle span per tile row / slab row
 constexpr int kATileBytes = kBM * kRowBytes;
 constexpr int kBTileBytes = kBN * kRowBytes;
@@ -44,6 +54,8 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+static_assert(kStagesPair * (kATileBytes + kBTileBytes / 2) <= kStages * kStageBytes,
+              "pair ring must fit the same shared-memory budget");
 
 constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
 constexpr float kLog2e = 1.4426950408889634f;
@@ -51,7 +63,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2 };
 
 struct GemmParams {
-  int tiles_m, tiles_n, num_kb;
+  int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
   void* out;           // STATS: logit buffer (nullable); STORE: dH; ACCUM: dW
   int64_t ld_out;      // row stride of out, elements
@@ -64,9 +76,27 @@ struct GemmParams {
   const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
   const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
+  int ksplit = 1;      // split of the K range into ksplit contiguous parts (>= 1)
+  int64_t split_stride = 0;  // ACCUM with ksplit > 1: elements between the parts' outputs
   int* status;         // device status word
   long long spin_limit;
 };
+
+// Work unit u covers output tile (u mod tiles) and K-part (u div tiles); the
+// host guarantees every part is non-empty.
+struct UnitRange {
+  int tile, ks, kb0, kb1;
+};
+__device__ __forceinline__ UnitRange unit_range(int u, const GemmParams& p) {
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int kbs = (p.num_kb + p.ksplit - 1) / p.ksplit;
+  UnitRange r;
+  r.tile = u % tiles;
+  r.ks = u / tiles;
+  r.kb0 = r.ks * kbs;
+  r.kb1 = min(p.num_kb, r.kb0 + kbs);
+  return r;
+}
 
 struct Ctl {
   int* status;
@@ -134,24 +164,30 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename Elem, int A_MN, int B_MN, int EPI>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int kCtas = PAIR ? 2 : 1;
+  constexpr int kNS = PAIR ? kStagesPair : kStages;   // ring depth
+  constexpr int kBRows = kBN / kCtas;                 // B rows staged by this CTA
+  constexpr int kBBytes = kBRows * kRowBytes;
+  constexpr int kSBytes = kATileBytes + kBBytes;      // this CTA's stage bytes
   constexpr int kEB = ElemTraits<Elem>::kBytes;
   constexpr int kBKe = kRowBytes / kEB;       // K elements per stage (64 / 32)
   constexpr int kUmmaK = 32 / kEB;            // K per MMA instruction (16 / 8)
   constexpr int kKSteps = kBKe / kUmmaK;      // 4
   constexpr int kMNe = kRowBytes / kEB;       // MN elements per MN-major slab
   constexpr int kSlabBytes = kBKe * kRowBytes;
-  constexpr uint32_t kIdesc = idesc_dense(ElemTraits<Elem>::kFmt, kBM, kBN, A_MN, B_MN);
+  constexpr uint32_t kIdesc =
+      idesc_dense(ElemTraits<Elem>::kFmt, kBM * kCtas, kBN, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty_bar = full_bar + kStages;
-  uint64_t* tfull_bar = empty_bar + kStages;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kNS * kSBytes);
+  uint64_t* empty_bar = full_bar + kNS;
+  uint64_t* tfull_bar = empty_bar + kNS;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -159,16 +195,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int total_tiles = p.tiles_m * p.tiles_n;
+  const int total_tiles = p.tiles_m * p.tiles_n * p.ksplit;  // work units
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // CTA rank within the pair
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 4 * 32);
+      mbar_init(&tempty_bar[b], 4 * kCtas);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -179,11 +219,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 5) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
     tc_fence_before();
   }
   __syncthreads();
+  if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const Ctl ctl{p.status, p.spin_limit, abort_flag};
@@ -193,55 +239,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       uint32_t issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < total_tiles && ok; t += units) {
+        const UnitRange ur = unit_range(t, p);
         int tm, tn;
-        tile_coords(t, p, tm, tn);
-        const int m0 = tm * kBM, n0 = tn * kBN;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          const uint32_t s = issued % kStages;
-          const uint32_t ph = (issued / kStages) & 1u;
+        tile_coords(ur.tile, p, tm, tn);
+        const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;  // this CTA's A rows
+        const int n0 = tn * kBN + static_cast<int>(rank) * kBRows;        // this CTA's B rows
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
+          const uint32_t s = issued % kNS;
+          const uint32_t ph = (issued / kNS) & 1u;
           if (!wait_bar(&empty_bar[s], ph ^ 1u, ctl)) {
             ok = false;
             break;
           }
-          uint8_t* a_s = smem + s * kStageBytes;
+          uint8_t* a_s = smem + s * kSBytes;
           uint8_t* b_s = a_s + kATileBytes;
-          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
+          const uint32_t fb = PAIR ? mapa_shared(&full_bar[s], 0) : 0u;
           const int k0 = kb * kBKe;
-          if (A_MN) {
 #pragma unroll
-            for (int sl = 0; sl < kBM / kMNe; ++sl)
-              tma_load_2d(&tmA, &full_bar[s], a_s + sl * kSlabBytes, m0 + sl * kMNe, k0);
-          } else {
-            tma_load_2d(&tmA, &full_bar[s], a_s, k0, m0);
+          for (int sl = 0; sl < (A_MN ? kBM / kMNe : 1); ++sl) {
+            void* dst = a_s + sl * kSlabBytes;
+            const int x = A_MN ? m0 + sl * kMNe : k0, y = A_MN ? k0 : m0;
+            if (PAIR) tma_load_2d_pair(&tmA, fb, dst, x, y);
+            else tma_load_2d(&tmA, &full_bar[s], dst, x, y);
           }
-          if (B_MN) {
 #pragma unroll
-            for (int sl = 0; sl < kBN / kMNe; ++sl)
-              tma_load_2d(&tmB, &full_bar[s], b_s + sl * kSlabBytes, n0 + sl * kMNe, k0);
-          } else {
-            tma_load_2d(&tmB, &full_bar[s], b_s, k0, n0);
+          for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
+            void* dst = b_s + sl * kSlabBytes;
+            const int x = B_MN ? n0 + sl * kMNe : k0, y = B_MN ? k0 : n0;
+            if (PAIR) tma_load_2d_pair(&tmB, fb, dst, x, y);
+            else tma_load_2d(&tmB, &full_bar[s], dst, x, y);
           }
           ++issued;
         }
       }
-      if (!ok) {
+      if (!ok && leader) {
         // Let the copies already issued land before the CTA exits.
         Ctl drain{p.status, p.spin_limit, abort_flag};
         volatile int no_abort = 0;
         drain.abort_flag = &no_abort;
-        const uint32_t first = issued > kStages ? issued - kStages : 0;
+        const uint32_t first = issued > kNS ? issued - kNS : 0;
         for (uint32_t n = first; n < issued; ++n)
-          wait_bar(&full_bar[n % kStages], (n / kStages) & 1u, drain);
+          wait_bar(&full_bar[n % kNS], (n / kNS) & 1u, drain);
       }
     }
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t consumed = 0, local = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+      for (int t = unit; t < total_tiles && ok; t += units, ++local) {
         const uint32_t buf = local & 1u;
         const uint32_t aph = (local >> 1) & 1u;
         if (!wait_bar(&tempty_bar[buf], aph ^ 1u, ctl)) {
@@ -250,15 +299,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * kBN;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          const uint32_t s = consumed % kStages;
-          const uint32_t ph = (consumed / kStages) & 1u;
+        const UnitRange ur = unit_range(t, p);
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
+          const uint32_t s = consumed % kNS;
+          const uint32_t ph = (consumed / kNS) & 1u;
           if (!wait_bar(&full_bar[s], ph, ctl)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+          const uint32_t a_addr = smem_u32(smem + s * kSBytes);
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
           for (int j = 0; j < kKSteps; ++j) {
@@ -268,22 +318,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t bd = B_MN ? sdesc_sw128(b_addr + j * (kUmmaK / 8) * 1024,
                                                    kSlabBytes, 1024)
                                      : sdesc_sw128(b_addr + j * 32, 16, 1024);
-            if (kEB == 2)
-              umma_f16(d_tmem, ad, bd, kIdesc, (kb | j) != 0);
-            else
-              umma_tf32(d_tmem, ad, bd, kIdesc, (kb | j) != 0);
+            const uint32_t acc = (kb != ur.kb0 || j != 0) ? 1u : 0u;
+            if (PAIR) {
+              if (kEB == 2) umma_f16_pair(d_tmem, ad, bd, kIdesc, acc);
+              else umma_tf32_pair(d_tmem, ad, bd, kIdesc, acc);
+            } else {
+              if (kEB == 2) umma_f16(d_tmem, ad, bd, kIdesc, acc);
+              else umma_tf32(d_tmem, ad, bd, kIdesc, acc);
+            }
           }
-          umma_commit(&empty_bar[s]);  // frees the smem stage when these MMAs finish
+          // frees the smem stage (in both CTAs of a pair) when these MMAs finish
+          if (PAIR) umma_commit_pair(&empty_bar[s], 0x3);
+          else umma_commit(&empty_bar[s]);
           ++consumed;
         }
         if (!ok) break;
-        umma_commit(&tfull_bar[buf]);  // accumulator ready for the epilogue
+        // accumulator ready for the epilogue(s)
+        if (PAIR) umma_commit_pair(&tfull_bar[buf], 0x3);
+        else umma_commit(&tfull_bar[buf]);
       }
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is released.
         volatile int no_abort = 0;
         Ctl drain{p.status, p.spin_limit, &no_abort};
-        umma_commit(drain_bar);
+        if (PAIR) umma_commit_pair(drain_bar, 0x1);
+        else umma_commit(drain_bar);
         wait_bar(drain_bar, 0, drain);
       }
     }
@@ -293,16 +352,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = warp * 32 + lane;  // accumulator row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     uint32_t local = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+    // The accumulator stage is released with one arrival per warp on the
+    // leader CTA's barrier (a remote arrive from the peer CTA of a pair).
+    const uint32_t tempty_cluster0 = PAIR ? mapa_shared(&tempty_bar[0], 0) : 0u;
+    const uint32_t tempty_cluster1 = PAIR ? mapa_shared(&tempty_bar[1], 0) : 0u;
+    auto release = [&](uint32_t buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(buf ? tempty_cluster1 : tempty_cluster0);
+        else mbar_arrive(&tempty_bar[buf]);
+      }
+    };
+    for (int t = unit; t < total_tiles; t += units, ++local) {
+      const UnitRange ur = unit_range(t, p);
       int tm, tn;
-      tile_coords(t, p, tm, tn);
+      tile_coords(ur.tile, p, tm, tn);
       const uint32_t buf = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
       if (!wait_bar(&tfull_bar[buf], aph, ctl)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_base + buf * kBN;
-      const int grow = tm * kBM + r;
+      const int grow = tm * kBM * kCtas + static_cast<int>(rank) * kBM + r;
       const bool rv = grow < p.rows_valid;
       const int col0 = tn * kBN;
 
@@ -332,10 +404,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           tmem_ld32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (c == kBN / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(&tempty_bar[buf]);
-          }
+          if (c == kBN / 32 - 1) release(buf);
           const int cb = col0 + c * 32;
           const int nvalid = p.cols_valid - cb;  // columns < V in this slab
           float cm = -INFINITY;
@@ -385,10 +454,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           tmem_ld32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (c == kBN / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(&tempty_bar[buf]);
-          }
+          if (c == kBN / 32 - 1) release(buf);
           if (!rv) continue;
           const int cb = col0 + c * 32;
           if (EPI == EPI_STORE) {
@@ -403,7 +469,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           } else {  // EPI_ACCUM, fp32 out
-            float* orow = static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+            float* orow = static_cast<float*>(p.out) + ur.ks * p.split_stride +
+                          static_cast<int64_t>(grow) * p.ld_out;
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
               if (cb + g * 4 < p.cols_valid) {
@@ -427,9 +494,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   __syncthreads();
+  if (PAIR) cluster_sync();  // neither CTA of a pair leaves while the other still works
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

@@ -394,6 +394,25 @@ __global__ void round_tf32_kernel(const float* __restrict__ src, int64_t ld_src,
   }
 }
 
+// out = sum over parts s = 0..S-1 of part[s] (fixed order), converted to Elem;
+// rows x cols values, part slices `slice` elements apart, row stride ld.
+template <typename Elem>
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int64_t slice,
+                                     Elem* __restrict__ out, int64_t n) {
+  const int64_t nv = n >> 2;  // n is a multiple of 8 (rows of d, d % 8 == 0)
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = reinterpret_cast<const float4*>(part)[i];
+    for (int s = 1; s < S; ++s) {
+      const float4 b = reinterpret_cast<const float4*>(part + s * slice)[i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    const float f[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[i * 4 + k] = from_f<Elem>(f[k]);
+  }
+}
+
 __global__ void fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
