@@ -326,7 +326,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
       return KL_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const int tiles = gp.tiles_m * gp.tiles_n;
+  const int tiles = gp.tiles_m * gp.tiles_n * gp.ksplit;  // work units
   const int units = PAIR ? sms / 2 : sms;  // CTA pairs or CTAs, one CTA per SM
   const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};

@@ -58,6 +58,10 @@ static_assert(kStagesPair * (kATileBytes + kBTileBytes / 2) <= kStages * kStageB
               "pair ring must fit the same shared-memory budget");
 
 constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
+// Bound of the waits that drain in-flight copies and MMAs after an abort.  It
+// does not shrink with the caller's spin limit: those copies and MMAs always
+// finish on their own, and the CTA must not leave before they do.
+constexpr long long kDrainLimit = 1LL << 31;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2 };
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok && leader) {
         // Let the copies already issued land before the CTA exits.
-        Ctl drain{p.status, p.spin_limit, abort_flag};
+        Ctl drain{p.status, kDrainLimit, abort_flag};
         volatile int no_abort = 0;
         drain.abort_flag = &no_abort;
         const uint32_t first = issued > kNS ? issued - kNS : 0;
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is released.
         volatile int no_abort = 0;
-        Ctl drain{p.status, p.spin_limit, &no_abort};
+        Ctl drain{p.status, kDrainLimit, &no_abort};
         if (PAIR) umma_commit_pair(drain_bar, 0x1);
         else umma_commit(drain_bar);
         wait_bar(drain_bar, 0, drain);
