@@ -42,13 +42,48 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kernels", choices=["kernels", "reference"])
-    ap.add_argument("--N", type=int, default=4096)
+    ap.add_argument("--workload", default="offline_topk",
+                    choices=["offline_topk", "full_vocab", "packed_long", "scaling"])
+    ap.add_argument("--N", type=int, default=0, help="tokens per GPU (0 = the workload's own)")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=0,
                     help="tokens in the oracle sample (0 = sized to ~10 s)")
     return ap.parse_args()
+
+
+WORKLOADS = {
+    "offline_topk": WORKLOAD,
+    "full_vocab": ("full-vocab recompute: N=8192, d=3072, teacher d_t=4096, V=128256, bf16 "
+                   "hiddens N(0,1), heads N(0,0.02^2); teacher logits recomputed per chunk; T=2"),
+    "packed_long": ("packed long context: N=32768 packed documents (lengths U[512,4096]), 5% of "
+                    "positions masked; d=3072, V=128256, bf16, K=64 cache as offline top-K; T=1"),
+    "scaling": ("output-head scaling sweep: offline top-K cache workload at the given N "
+                "(4096/16384/65536/262144); d=3072, V=128256, bf16, K=64; T=1"),
+}
+
+
+def make_workload(wl, args, dev, rank):
+    seed_shift = rank * 1000
+    if args.workload == "offline_topk":
+        return wl.offline_topk(device=dev, N=args.N or 4096, seed=1 + seed_shift)
+    if args.workload == "full_vocab":
+        return wl.full_vocab(device=dev, N=args.N or 8192, seed=2 + seed_shift)
+    if args.workload == "packed_long":
+        return wl.packed_long(device=dev, N=args.N or 32768, seed=3 + seed_shift)
+    return wl.scaling(args.N or 262144, device=dev, seed=4 + seed_shift)
+
+
+def problem_kwargs(w, chunk, override=None):
+    o = override or {}
+    kw = dict(T=w.T, mask=o.get("mask", w.mask), chunk_tokens=chunk)
+    if w.mode == "topk":
+        kw.update(topk_idx=o.get("topk_idx", w.topk_idx), topk_logit=o.get("topk_logit", w.topk_logit),
+                  teacher_lse=o.get("teacher_lse", w.teacher_lse))
+    else:
+        kw.update(Ht=o.get("Ht", w.Ht), Wt=w.Wt)
+    return kw
 
 
 def dist_setup(args):
@@ -130,10 +165,10 @@ def gpu_arm(args):
     dev = torch.device("cuda", local)
     if ws > 1:
         dist.init_process_group("nccl", device_id=dev)
-    w = wl.offline_topk(device=dev, N=args.N, seed=1 + rank)
+    w = make_workload(wl, args, dev, rank)
+    args.N = w.N
     torch.cuda.empty_cache()  # drop the teacher-cache generator's temporaries
-    kw = dict(T=w.T, topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse,
-              chunk_tokens=args.chunk)
+    kw = problem_kwargs(w, args.chunk)
     prob, keep = ops.make_problem(w.H, w.W, **kw)
     ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
     torch.cuda.synchronize()
@@ -185,21 +220,18 @@ def gpu_arm(args):
     # ---- end to end through the public API: pinned host inputs in, loss out
     e2e = None
     if not args.no_e2e:
-        hH = w.H.cpu().pin_memory()
-        hidx = w.topk_idx.cpu().pin_memory()
-        hval = w.topk_logit.cpu().pin_memory()
-        hlse = w.teacher_lse.cpu().pin_memory()
+        # per-step inputs: hidden states and the teacher side (cache or teacher
+        # hidden states) and the mask; the heads stay resident (parameters)
+        names = ["H", "mask", "topk_idx", "topk_logit", "teacher_lse", "Ht"]
+        host = {k: getattr(w, k).cpu().pin_memory() for k in names if getattr(w, k) is not None}
+        devb = {k: torch.empty_like(getattr(w, k)) for k in host}
         hloss = torch.empty((), dtype=torch.float32).pin_memory()
-        dHin, didx, dval, dlse = (torch.empty_like(w.H), torch.empty_like(w.topk_idx),
-                                  torch.empty_like(w.topk_logit), torch.empty_like(w.teacher_lse))
-        prob2, keep2 = ops.make_problem(dHin, w.W, T=w.T, topk_idx=didx, topk_logit=dval,
-                                        teacher_lse=dlse, chunk_tokens=args.chunk)
+        kw2 = problem_kwargs(w, args.chunk, override=devb)
+        prob2, keep2 = ops.make_problem(devb["H"], w.W, **kw2)
 
         def e2e_step():
-            dHin.copy_(hH, non_blocking=True)
-            didx.copy_(hidx, non_blocking=True)
-            dval.copy_(hval, non_blocking=True)
-            dlse.copy_(hlse, non_blocking=True)
+            for k in host:
+                devb[k].copy_(host[k], non_blocking=True)
             _lib.check(_lib.kl_fwd_bwd(prob2, workspace.data_ptr(), ws_bytes, 1.0,
                                        loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(), 0,
                                        stream), "kl_fwd_bwd")
@@ -216,7 +248,7 @@ def gpu_arm(args):
         ems = e0.elapsed_time(e1)
         if ws > 1:
             ems = max_over_ranks(ems)
-        h2d = sum(t.numel() * t.element_size() for t in (hH, hidx, hval, hlse))
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
         e2e = {"value": ws * args.N * args.steps / (ems / 1e3),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
 
@@ -227,7 +259,7 @@ def gpu_arm(args):
         return
 
     peaks, peak_src = measured_peaks()
-    N, d, V = args.N, 3072, 128256
+    N, d, V = args.N, w.d, w.V
     tok_s = ws * N * args.steps / (ms / 1e3)
     dom = max(prof, key=lambda p: p["total_ms"]) if prof else None
     roof = None
@@ -248,7 +280,9 @@ def gpu_arm(args):
             roof = {"kernel": dom["name"], "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
-    step_flops = 6.0 * N * d * V
+    # algorithmic tensor work per step: logits, dH and dW contractions (6 N d V),
+    # plus the teacher logits (2 N d_t V) in the teacher-hidden mode
+    step_flops = 6.0 * N * d * V + (2.0 * N * w.d_t * V if w.mode == "hidden" else 0.0)
     step_tflops = step_flops * args.steps / (ms / 1e3) / 1e12
     kernels = {p["name"]: {"launches": p["launches"], "ms": round(p["total_ms"], 3),
                            "share": round(p["total_ms"] / sum(q["total_ms"] for q in prof), 4)}
@@ -258,7 +292,9 @@ def gpu_arm(args):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init heads and teacher cache)",
-        "config": {"workload": WORKLOAD, "N_per_gpu": N, "d": d, "V": V, "K": 64, "T": 1.0,
+        "config": {"workload": WORKLOADS[args.workload], "N_per_gpu": N, "d": d, "V": V,
+                   "K": w.K or None, "d_t": w.d_t if w.mode == "hidden" else None, "T": w.T,
+                   "masked_tokens": int((w.mask == 0).sum().item()) if w.mask is not None else 0,
                    "chunk_tokens": args.chunk or min(4096, N),
                    "l2": "inputs larger than L2 (W 0.79 GB, logit chunk 1.05 GB); no flush",
                    "parallelism": f"weak-scaling token shards x{ws}, no data-path collective"},
@@ -273,6 +309,8 @@ def gpu_arm(args):
     }
     if not args.no_cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
+    if args.workload != "offline_topk":
+        line["metric"] = METRIC + f" [{args.workload}]"
     print(json.dumps(line), flush=True)
 
 
@@ -282,8 +320,13 @@ def _oracle_sample(w, n_tokens):
     import oracle
 
     sl = slice(0, n_tokens)
-    return oracle.kl_loss(w.H[sl], w.W, T=w.T, mode="topk", topk_idx=w.topk_idx[sl],
-                          topk_logit=w.topk_logit[sl], teacher_lse=w.teacher_lse[sl])
+    kw = dict(T=w.T, mode=w.mode, mask=None if w.mask is None else w.mask[sl])
+    if w.mode == "topk":
+        kw.update(topk_idx=w.topk_idx[sl], topk_logit=w.topk_logit[sl],
+                  teacher_lse=None if w.teacher_lse is None else w.teacher_lse[sl])
+    else:
+        kw.update(Ht=w.Ht[sl], Wt=w.Wt)
+    return oracle.kl_loss(w.H[sl], w.W, **kw)
 
 
 def _cores():
@@ -298,18 +341,20 @@ def _cores():
     return os.cpu_count()
 
 
-def cpu_baseline(w, n_tokens=0):
-    """fp64 oracle throughput on the host cores over a bounded token sample."""
-    import numpy as np
-
-    Wd = w.W.cpu()
+def cpu_baseline(w, n_tokens=0, target_s=10.0):
+    """fp64 oracle throughput on the host cores over a bounded token sample,
+    sized from two short probes to about target_s seconds of CPU work."""
     sample = w.to("cpu")
-    sample.W = Wd
-    t0 = time.time()
-    _oracle_sample(sample, 8)
-    t_probe = time.time() - t0
     if n_tokens <= 0:
-        n_tokens = int(np.clip(8 * 10.0 / max(t_probe, 1e-3), 8, 512))
+        t0 = time.time()
+        _oracle_sample(sample, 8)
+        t8 = time.time() - t0
+        t0 = time.time()
+        _oracle_sample(sample, 40)
+        t40 = time.time() - t0
+        per_token = max((t40 - t8) / 32, 1e-6)
+        fixed = max(t8 - 8 * per_token, 0.0)
+        n_tokens = int(min(max((target_s - fixed) / per_token, 16), 4096, w.N))
     t0 = time.time()
     _oracle_sample(sample, n_tokens)
     dt = time.time() - t0
@@ -328,7 +373,8 @@ def reference_arm(args):
     from chunked_kl_loss_tma_b200 import workloads as wl
 
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    w = wl.offline_topk(device=dev, N=args.N, seed=1).to("cpu")
+    w = make_workload(wl, args, dev, 0).to("cpu")
+    args.N = w.N
     per_step = args.cpu_sample or 16
     for _ in range(max(args.warmup, 3)):
         _oracle_sample(w, 2)
@@ -337,12 +383,13 @@ def reference_arm(args):
         _oracle_sample(w, per_step)
     dt = time.time() - t0
     v = per_step * args.steps / dt
+    metric = METRIC + ("" if args.workload == "offline_topk" else f" [{args.workload}]")
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
+        "impl": "reference", "metric": metric, "value": round(v, 3), "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "N_per_gpu": args.N,
+        "config": {"workload": WORKLOADS[args.workload], "N_per_gpu": w.N,
                    "sample_per_step": f"{per_step} tokens (fp64 oracle on host cores)"},
         "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": _cores(),
                          "kind": "oracle",

@@ -85,7 +85,8 @@ EncodeTiledFn encode_fn() {
 // 2-D map over a row-major matrix [rows][inner] with the given row stride,
 // 128-byte swizzle, zero fill outside the extents.
 bool make_map(CUtensorMap* m, const void* base, int dtype, uint64_t inner, uint64_t rows,
-              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, rows};
@@ -95,9 +96,17 @@ bool make_map(CUtensorMap* m, const void* base, int dtype, uint64_t inner, uint6
   const CUresult r =
       fn(m, dtype == KL_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
          2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Output map of the GEMM epilogue: 32 x 32 boxes staged in shared memory with
+// 64-byte rows (bf16, 64-byte swizzle) or 128-byte rows (fp32, 128-byte swizzle).
+bool make_out_map(CUtensorMap* m, const void* base, int dtype, uint64_t inner, uint64_t rows,
+                  uint64_t row_stride_bytes) {
+  return make_map(m, base, dtype, inner, rows, row_stride_bytes, 32, 32,
+                  dtype == KL_DTYPE_BF16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // ------------------------------------------------------------------ profiling
@@ -294,7 +303,8 @@ Plan make_plan(const kl_problem* p, int entry) {
     pl.ksplit_dh = choose_ksplit(cdiv(pl.C, 2 * kBM) * cdiv(p->d, kBN), cdiv(p->V, 64),
                                  max_units_hint());
     if (pl.ksplit_dh > 1)
-      pl.off_dhp = take(static_cast<size_t>(pl.ksplit_dh) * pl.C * p->d * 4);
+      pl.off_dhp = take(static_cast<size_t>(pl.ksplit_dh) * cdiv(pl.C, 2 * kBM) * 2 * kBM *
+                        p->d * 4);
   }
   if (pl.eb == 4) {
     const int64_t dmax = (pl.hidden && p->d_t > p->d) ? p->d_t : p->d;
@@ -315,7 +325,7 @@ Plan make_plan(const kl_problem* p, int entry) {
 // ------------------------------------------------------------------ launches
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
-                const CUtensorMap& mb, GemmParams gp, double flops) {
+                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
   auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
@@ -346,7 +356,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, gp);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
@@ -402,19 +412,23 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
     KL_TRY(launch_round(c, reinterpret_cast<const float*>(xc), dx, xr, dx, Cn, dx));
     xc = reinterpret_cast<const uint8_t*>(xr);
   }
+  CUtensorMap mc;
   if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
       !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2))
     return KL_ERR_CUDA;
+  if (out != nullptr) {
+    if (!make_out_map(&mc, out, p->dtype, p->V, Cn, c.pl.Vp * sizeof(Elem))) return KL_ERR_CUDA;
+  } else {
+    mc = mb;  // statistics only: the output map is not used
+  }
   GemmParams gp{};
   gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
   gp.tiles_n = c.pl.tiles_v;
   gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
   gp.m_fastest = 1;
-  gp.out = out;
-  gp.ld_out = c.pl.Vp;
+  gp.store = out != nullptr;
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
-  gp.cols_store = static_cast<int>(c.pl.Vp);
   gp.scale = c.invT;
   gp.partials = partials;
   gp.sidx = sidx;
@@ -422,7 +436,7 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.ktop = ktop;
   gp.status = &c.sc->status;
   gp.spin_limit = spin_limit();
-  return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, gp,
+  return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, mc, gp,
                                                2.0 * Cn * p->V * dx);
 }
 
@@ -447,42 +461,40 @@ int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* d
   KL_TRY(launch_transpose(c, dS, c.pl.Vp, sT, Cp, Cn, V));
   KL_TRY(launch_transpose(c, hc, d, hT, Cp, Cn, d));
   {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mc;
     if (!make_map(&ma, dS, p->dtype, V, Cn, c.pl.Vp * 4, 32, kBM) ||
-        !make_map(&mb, wT, p->dtype, V, d, c.pl.Vp * 4, 32, kBN / 2))
+        !make_map(&mb, wT, p->dtype, V, d, c.pl.Vp * 4, 32, kBN / 2) ||
+        !make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
       return KL_ERR_CUDA;
     GemmParams gp{};
     gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(V, 32));
     gp.m_fastest = 1;
-    gp.out = static_cast<float*>(dH) + c0 * d;
-    gp.ld_out = d;
     gp.rows_valid = static_cast<int>(Cn);
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<float, 0, 0, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+    KL_TRY((launch_gemm<float, 0, 0, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                    2.0 * Cn * V * d)));
   }
   {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mc;
     if (!make_map(&ma, sT, p->dtype, Cn, V, Cp * 4, 32, kBM) ||
-        !make_map(&mb, hT, p->dtype, Cn, d, Cp * 4, 32, kBN / 2))
+        !make_map(&mb, hT, p->dtype, Cn, d, Cp * 4, 32, kBN / 2) ||
+        !make_out_map(&mc, dW, KL_DTYPE_F32, d, V, d * 4))
       return KL_ERR_CUDA;
     GemmParams gp{};
     gp.tiles_m = static_cast<int>(cdiv(V, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(Cn, 32));
     gp.m_fastest = 0;
-    gp.out = dW;
-    gp.ld_out = d;
     gp.rows_valid = static_cast<int>(V);
     gp.cols_valid = static_cast<int>(d);
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<float, 0, 0, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, gp,
+    KL_TRY((launch_gemm<float, 0, 0, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
                                                    2.0 * Cn * V * d)));
   }
   return KL_OK;
@@ -510,7 +522,6 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(p->V, kBKe));
     gp.m_fastest = 1;
-    gp.ld_out = d;
     gp.rows_valid = static_cast<int>(Cn);
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
@@ -519,42 +530,50 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     if (ks > c.pl.ksplit_dh) ks = c.pl.ksplit_dh;
     if (ks > 1) {
       float* part = reinterpret_cast<float*>(c.ws + c.pl.off_dhp);
+      // Each K-part owns a slice padded to whole 256-row tiles: output boxes
+      // that overhang the chunk's last row land in the part's own padding,
+      // never in the next part's rows.
+      const int64_t rows_pad = cdiv(Cn, 2 * kBM) * 2 * kBM;
       gp.ksplit = ks;
-      gp.split_stride = Cn * d;
-      gp.out = part;
+      gp.split_rows = static_cast<int>(rows_pad);
       gp.beta = 0;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+      CUtensorMap mc;
+      if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
+        return KL_ERR_CUDA;
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
       LaunchScope ls("splitk_reduce", c.st, 0, (4.0 * ks + sizeof(Elem)) * Cn * d);
       splitk_reduce_kernel<Elem><<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(
-          part, ks, Cn * d, static_cast<Elem*>(dH) + c0 * d, Cn * d);
+          part, ks, rows_pad * d, static_cast<Elem*>(dH) + c0 * d, Cn * d);
       KL_TRY(cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA);
     } else {
-      gp.out = static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem);
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, gp,
+      CUtensorMap mc;
+      if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
+                        d * sizeof(Elem)))
+        return KL_ERR_CUDA;
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
     }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
   {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mc;
     const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * d * sizeof(Elem);
     if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
-        !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe))
+        !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe) ||
+        !make_out_map(&mc, dW, KL_DTYPE_F32, d, p->V, d * 4))
       return KL_ERR_CUDA;
     GemmParams gp{};
     gp.tiles_m = static_cast<int>(cdiv(p->V, 2 * kBM));
     gp.tiles_n = static_cast<int>(cdiv(d, kBN));
     gp.num_kb = static_cast<int>(cdiv(Cn, kBKe));
     gp.m_fastest = 0;
-    gp.out = dW;
-    gp.ld_out = d;
     gp.rows_valid = static_cast<int>(p->V);
     gp.cols_valid = static_cast<int>(d);
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, gp,
+    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
                                                   2.0 * Cn * p->V * d)));
   }
   return KL_OK;

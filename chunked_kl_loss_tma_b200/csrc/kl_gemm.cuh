@@ -53,9 +53,14 @@ constexpr int kBTileBytes = kBN * kRowBytes;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-static_assert(kStagesPair * (kATileBytes + kBTileBytes / 2) <= kStages * kStageBytes,
+constexpr int kRingBytes = kStages * kStageBytes;          // 192 KB operand ring
+constexpr int kBarrierRegion = 1024;                        // barriers, TMEM slot, flags
+constexpr int kStageOutBytes = 4096;                        // one 32 x 32 fp32 output box
+constexpr int kStagingBytes = 4 * 2 * kStageOutBytes;       // 4 epilogue warps x 2 buffers
+constexpr int kGemmSmemBytes = 1024 /*align*/ + kRingBytes + kBarrierRegion + kStagingBytes;
+static_assert(kStagesPair * (kATileBytes + kBTileBytes / 2) <= kRingBytes,
               "pair ring must fit the same shared-memory budget");
+static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
 
 constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
 // Bound of the waits that drain in-flight copies and MMAs after an abort.  It
@@ -69,11 +74,9 @@ enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2 };
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
-  void* out;           // STATS: logit buffer (nullable); STORE: dH; ACCUM: dW
-  int64_t ld_out;      // row stride of out, elements
+  int store;           // STATS: store s~ through the output map (0 = statistics only)
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
-  int cols_store;      // STATS: columns written to the logit buffer (padded V)
   float scale;         // STATS: 1 / T
   int beta;            // ACCUM: 0 overwrite, 1 accumulate
   float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross, 0)
@@ -81,7 +84,7 @@ struct GemmParams {
   const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
   int ksplit = 1;      // split of the K range into ksplit contiguous parts (>= 1)
-  int64_t split_stride = 0;  // ACCUM with ksplit > 1: elements between the parts' outputs
+  int split_rows = 0;  // ACCUM with ksplit > 1: output-map rows between the parts' outputs
   int* status;         // device status word
   long long spin_limit;
 };
@@ -171,7 +174,8 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                   const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kNS = PAIR ? kStagesPair : kStages;   // ring depth
   constexpr int kBRows = kBN / kCtas;                 // B rows staged by this CTA
@@ -189,7 +193,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kNS * kSBytes);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+  uint8_t* staging = smem + kRingBytes + kBarrierRegion;  // 1024-B aligned
   uint64_t* empty_bar = full_bar + kNS;
   uint64_t* tfull_bar = empty_bar + kNS;
   uint64_t* tempty_bar = tfull_bar + 2;
@@ -353,8 +358,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each warp stages its 32 rows x 32 columns of output in shared memory
+    // (two buffers, swizzled to match the output map) and one lane issues a TMA
+    // bulk store -- an fp32 add-reduction into global memory when accumulating.
     const int r = warp * 32 + lane;  // accumulator row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    uint8_t* stg = staging + warp * 2 * kStageOutBytes;
+    uint32_t nbox = 0;  // output boxes this warp has staged
     uint32_t local = 0;
     // The accumulator stage is released with one arrival per warp on the
     // leader CTA's barrier (a remote arrive from the peer CTA of a pair).
@@ -368,6 +378,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else mbar_arrive(&tempty_bar[buf]);
       }
     };
+    // Stage v * scale (32 values of this thread's row) and store the warp's box
+    // at output column x, output-map row y (rows past row_end are not written).
+    auto store_box = [&](const uint32_t(&v)[32], float scale, int x, int y, bool fp32_out,
+                         bool reduce, bool issue) {
+      uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
+      ++nbox;
+      if (lane == 0) bulk_wait_read_1();  // the store that last used sb has read it
+      __syncwarp();
+      if (fp32_out) {  // 128-byte rows, 128-byte swizzle: chunk j at j ^ (row & 7)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 q = make_float4(__uint_as_float(v[4 * j]) * scale,
+                                       __uint_as_float(v[4 * j + 1]) * scale,
+                                       __uint_as_float(v[4 * j + 2]) * scale,
+                                       __uint_as_float(v[4 * j + 3]) * scale);
+          *reinterpret_cast<float4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) = q;
+        }
+      } else {  // bf16: 64-byte rows, 64-byte swizzle: chunk j at j ^ ((row >> 1) & 3)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float f[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[8 * j + i]) * scale;
+          store_vec<__nv_bfloat16>(
+              reinterpret_cast<__nv_bfloat16*>(sb + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)),
+              f);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && issue) {
+        if (reduce) tma_reduce_add_2d(&tmC, sb, x, y);
+        else tma_store_2d(&tmC, sb, x, y);
+        bulk_commit();
+      }
+    };
+    constexpr bool kElemF32 = sizeof(Elem) == 4;
     for (int t = unit; t < total_tiles; t += units, ++local) {
       const UnitRange ur = unit_range(t, p);
       int tm, tn;
@@ -378,8 +425,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_base + buf * kBN;
-      const int grow = tm * kBM * kCtas + static_cast<int>(rank) * kBM + r;
+      const int row0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM + warp * 32;
+      const int grow = row0 + lane;
       const bool rv = grow < p.rows_valid;
+      const bool warp_rows = row0 < p.rows_valid;  // any row of this warp's box exists
       const int col0 = tn * kBN;
 
       if (EPI == EPI_STATS) {
@@ -399,9 +448,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
-        Elem* orow = (p.out != nullptr && rv)
-                         ? static_cast<Elem*>(p.out) + static_cast<int64_t>(grow) * p.ld_out
-                         : nullptr;
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t v[32];
@@ -437,17 +483,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ++gi;
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
-          if (orow != nullptr) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (cb + g * 8 < p.cols_store) {
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[g * 8 + i]) * p.scale;
-                store_vec<Elem>(orow + cb + g * 8, f);
-              }
-            }
-          }
+          if (p.store && cb < p.cols_valid)
+            store_box(v, p.scale, cb, row0, kElemF32, false, warp_rows);
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
@@ -459,42 +496,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tbase + c * 32, v);
           tmem_ld_wait();
           if (c == kBN / 32 - 1) release(buf);
-          if (!rv) continue;
           const int cb = col0 + c * 32;
-          if (EPI == EPI_STORE) {
-            Elem* orow = static_cast<Elem*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (cb + g * 8 < p.cols_valid) {
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[g * 8 + i]);
-                store_vec<Elem>(orow + cb + g * 8, f);
-              }
-            }
-          } else {  // EPI_ACCUM, fp32 out
-            float* orow = static_cast<float*>(p.out) + ur.ks * p.split_stride +
-                          static_cast<int64_t>(grow) * p.ld_out;
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              if (cb + g * 4 < p.cols_valid) {
-                float4* o = reinterpret_cast<float4*>(orow + cb + g * 4);
-                float4 a = make_float4(__uint_as_float(v[g * 4 + 0]), __uint_as_float(v[g * 4 + 1]),
-                                       __uint_as_float(v[g * 4 + 2]), __uint_as_float(v[g * 4 + 3]));
-                if (p.beta) {
-                  const float4 old = *o;
-                  a.x += old.x;
-                  a.y += old.y;
-                  a.z += old.z;
-                  a.w += old.w;
-                }
-                *o = a;
-              }
-            }
-          }
+          if (cb >= p.cols_valid) continue;
+          if (EPI == EPI_STORE)
+            store_box(v, 1.f, cb, row0, kElemF32, false, warp_rows);
+          else  // EPI_ACCUM, fp32 out; K-part ks writes its own block of output rows
+            store_box(v, 1.f, cb, row0 + ur.ks * p.split_rows, true, p.beta != 0, warp_rows);
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // every output box has landed before exit
+    __syncwarp();
   }
 
   __syncthreads();
