@@ -93,6 +93,33 @@ def dist_setup(args):
     return ws, rank, local
 
 
+KERNEL_SOURCES = ["kl_gemm.cuh", "kl_ptx.cuh", "kl_rowops.cuh", "kl_api.cu"]
+
+
+def measured_traffic(workload, N):
+    """DRAM bytes per launch from the committed ncu summary of the same workload,
+    or {} when the kernel sources changed since the counters were taken."""
+    import hashlib
+    import re
+
+    if workload != "offline_topk" or N != 4096:
+        return {}
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "chunked_kl_loss_tma_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    src = h.hexdigest()[:16]
+    out = {}
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic_offline_topk_N4096.md")) as fh:
+            for m in re.finditer(r"^traffic-per-launch (\S+) (\d+) src=(\w+)$", fh.read(), re.M):
+                if m.group(3) == src:
+                    out[m.group(1)] = int(m.group(2))
+    except OSError:
+        pass
+    return out
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -171,19 +198,20 @@ def gpu_arm(args):
     kw = problem_kwargs(w, args.chunk)
     prob, keep = ops.make_problem(w.H, w.W, **kw)
     ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
-    torch.cuda.synchronize()
-    base_mem = torch.cuda.memory_allocated(dev)
-    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     dH = torch.empty_like(w.H)
     dW = torch.empty(w.W.shape, dtype=torch.float32, device=dev)
+    # extra HBM = everything allocated beyond inputs and gradients (the workspace)
+    torch.cuda.synchronize()
+    base_mem = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
 
     def step():
         _lib.check(_lib.kl_fwd_bwd(prob, workspace.data_ptr(), ws_bytes, 1.0, loss.data_ptr(),
                                    None, dH.data_ptr(), dW.data_ptr(), 0, stream), "kl_fwd_bwd")
 
-    torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
@@ -271,7 +299,7 @@ def gpu_arm(args):
             peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
             roof = {"kernel": dom["name"], "bound": "tensor", "achieved": round(achieved, 1),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "traffic": None,
+                    "traffic": measured_traffic(args.workload, N).get(dom["name"]),
                     "peak_source": f"{peak_src} sustained bf16 (kernel timed inside a long step)",
                     "avg_launch_ms": round(avg_s * 1e3, 4),
                     "flops_per_launch": per_launch_flops}
@@ -279,7 +307,8 @@ def gpu_arm(args):
             achieved = dom["bytes"] / max(dom["launches"], 1) / avg_s / 1e9
             roof = {"kernel": dom["name"], "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+                    "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": measured_traffic(args.workload, N).get(dom["name"])}
     # algorithmic tensor work per step: logits, dH and dW contractions (6 N d V),
     # plus the teacher logits (2 N d_t V) in the teacher-hidden mode
     step_flops = 6.0 * N * d * V + (2.0 * N * w.d_t * V if w.mode == "hidden" else 0.0)
