@@ -500,6 +500,49 @@ int gemm_grads_f32(Ctx& c, float* dS, int64_t c0, int64_t Cn, void* dH, float* d
   return KL_OK;
 }
 
+// Backward with known lse (split path, top-K mode): the recomputed logits tile
+// becomes dS in the GEMM epilogue and is stored to the chunk buffer.
+template <typename Elem>
+int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, const float* g_dev,
+                 float g_host) {
+  const kl_problem* p = c.p;
+  constexpr int kBKe = kRowBytes / sizeof(Elem);
+  const int64_t dx = p->d;
+  CUtensorMap ma, mb, mc;
+  const uint8_t* xc = static_cast<const uint8_t*>(p->H) + c0 * dx * sizeof(Elem);
+  if (sizeof(Elem) == 4) {  // tf32: round the chunk of hidden states first
+    float* xr = reinterpret_cast<float*>(c.ws + c.pl.off_xr);
+    KL_TRY(launch_round(c, reinterpret_cast<const float*>(xc), dx, xr, dx, Cn, dx));
+    xc = reinterpret_cast<const uint8_t*>(xr);
+  }
+  if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
+      !make_map(&mb, head_W(c), p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2) ||
+      !make_out_map(&mc, S, p->dtype, p->V, Cn, c.pl.Vp * sizeof(Elem)))
+    return KL_ERR_CUDA;
+  GemmParams gp{};
+  gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
+  gp.tiles_n = c.pl.tiles_v;
+  gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
+  gp.m_fastest = 1;
+  gp.store = 1;
+  gp.rows_valid = static_cast<int>(Cn);
+  gp.cols_valid = static_cast<int>(p->V);
+  gp.scale = c.invT;
+  gp.sidx = reinterpret_cast<const int*>(c.ws + c.pl.off_sidx);
+  gp.sq = reinterpret_cast<const float*>(c.ws + c.pl.off_sq);
+  gp.ktop = p->K;
+  gp.lse = lse_s + c0;
+  gp.rowinfo = reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo);
+  gp.mask = p->mask ? p->mask + c0 : nullptr;
+  gp.norm = &c.sc->norm;
+  gp.g_dev = g_dev;
+  gp.g_host = g_host;
+  gp.status = &c.sc->status;
+  gp.spin_limit = spin_limit();
+  return launch_gemm<Elem, 0, 0, EPI_DLOGITS, 1>("gemm_dlogits", c.st, c.sms, ma, mb, mc, gp,
+                                                 2.0 * Cn * p->V * dx);
+}
+
 template <typename Elem>
 int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta) {
   if (sizeof(Elem) == 4)
@@ -736,9 +779,7 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
     const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
     if (!c.pl.hidden) {
       KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, nullptr, nullptr, nullptr, 0,
-                               "gemm_logits_recompute"));
-      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
+      KL_TRY(gemm_dlogits<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
     } else {
       KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, nullptr, nullptr, nullptr, 0,
                                "gemm_logits_recompute"));

@@ -13,7 +13,11 @@
 //              the tile (gathered from the fp32 accumulator); optionally
 //              stores s~ = s / T to the chunk's logit buffer.
 //   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
-//   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, read-modify-write across chunks.
+//   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, add-reduced into dW across chunks.
+//   EPI_DLOGITS backward with the row lse already known (the split forward /
+//              backward path): dS = c (m exp(s~ - lse) - q [j in S]) formed from
+//              the fp32 accumulator and stored, with c = g / (n T) (0 on masked
+//              rows) -- no logits are stored and no separate dlogits pass runs.
 //
 // Two tile shapes: PAIR = 0, one CTA computes a 128 x 256 tile with
 // tcgen05.mma.cta_group::1; PAIR = 1, a cluster of two CTAs (one per SM)
@@ -69,7 +73,7 @@ constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
 constexpr long long kDrainLimit = 1LL << 31;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2 };
+enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3 };
 
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
@@ -83,6 +87,14 @@ struct GemmParams {
   const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
   const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
+  // DLOGITS: per-row lse (natural units), (m, .) per row, mask, and the scalars
+  // of c = g / (n T): the loss normaliser n, and g (device pointer or value)
+  const float* lse;
+  const float2* rowinfo;
+  const uint8_t* mask;
+  const float* norm;
+  const float* g_dev;
+  float g_host;
   int ksplit = 1;      // split of the K range into ksplit contiguous parts (>= 1)
   int split_rows = 0;  // ACCUM with ksplit > 1: output-map rows between the parts' outputs
   int* status;         // device status word
@@ -138,6 +150,13 @@ struct ElemTraits<float> {
   static constexpr int kBytes = 4;
   static constexpr uint32_t kFmt = 2;  // tf32
 };
+
+// Round-to-nearest onto the tf32 grid (for dS stored as an fp32 tf32 operand).
+__device__ __forceinline__ float round_tf32_dev(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
 
 __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm, int& tn) {
   if (p.m_fastest) {
@@ -488,6 +507,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
+      } else if (EPI == EPI_DLOGITS) {
+        float coef = 0.f, cm = 0.f, l2 = 0.f;
+        int gi = 0, gcol = 0x7fffffff;
+        const int* ri = nullptr;
+        const float* rq = nullptr;
+        if (rv) {
+          const bool keep = p.mask == nullptr || p.mask[grow] != 0;
+          const float g = p.g_dev != nullptr ? *p.g_dev : p.g_host;
+          const float n = *p.norm;
+          coef = (keep && n > 0.f) ? g / n * p.scale : 0.f;
+          cm = coef * p.rowinfo[grow].x;
+          l2 = p.lse[grow] * kLog2e;
+          ri = p.sidx + static_cast<int64_t>(grow) * p.ktop;
+          rq = p.sq + static_cast<int64_t>(grow) * p.ktop;
+          int lo = 0, hi = p.ktop;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(ri + mid) < col0) lo = mid + 1; else hi = mid;
+          }
+          gi = lo;
+          gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
+        }
+        const float s2 = p.scale * kLog2e;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (c == kBN / 32 - 1) release(buf);
+          const int cb = col0 + c * 32;
+          if (cb >= p.cols_valid) continue;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(v[i]) * s2;
+            v[i] = __float_as_uint(cm * ex2_approx(x - l2));
+          }
+          while (gcol < cb + 32) {  // subtract c q at the cached ids inside this slab
+            const int k = gcol - cb;
+            const float cq = coef * __ldg(rq + gi);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = (i == k) ? __float_as_uint(__uint_as_float(v[i]) - cq) : v[i];
+            ++gi;
+            gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
+          }
+          if (sizeof(Elem) == 4) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(round_tf32_dev(__uint_as_float(v[i])));
+          }
+          store_box(v, 1.f, cb, row0, kElemF32, false, warp_rows);
+        }
       } else {
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {

@@ -114,6 +114,26 @@ def test_offline_topk_4096_full_oracle_pass():
     _identities(w, out)
 
 
+def test_offline_topk_4096_split_forward_backward():
+    """kl_fwd then kl_bwd (backward recomputes the logits and forms dS in the
+    GEMM epilogue) against the oracle's sampled rows and the fused path."""
+    w = wl.offline_topk(device="cuda", seed=5)
+    kw = _kw(w)
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], **kw)
+    assert ops.status(f["workspace"]) == 0 and ops.status(b["workspace"]) == 0
+    fused = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
+    out = dict(row_loss=f["row_loss"], dH=b["dH"], dW=b["dW"], loss=f["loss"])
+    rows = _rows(w.N, None, n_random=16, seed=5)
+    _check_rows(w, out, rows, w.N)
+    _loss_is_mean_of_rows(out, w.N)
+    _identities(w, out)
+    assert abs(f["loss"].item() - fused["loss"].item()) <= 1e-5 * abs(fused["loss"].item())
+    for k in ("dH", "dW"):
+        a, c = b[k].double(), fused[k].double()
+        assert (a - c).abs().max().item() <= 2e-2 * c.abs().max().item(), k
+
+
 def test_full_vocab_8192_teacher_hidden():
     w = wl.full_vocab(device="cuda")
     out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w))
