@@ -37,6 +37,12 @@ Readings where the pages are silent (all restated in the design doc):
   R4 cache slot with index -1 is empty (contributes nothing); a row with no
      valid slot contributes 0; duplicate or out-of-range indices are errors.
   R5 frozen teacher head: no gradient flows to Ht or Wt.
+  R6 KL direction mixing (teacher-hidden mode only): the page's KL-direction
+     study (thelatestinai.com/papers/2606.20005, fourth abstract) names
+     token-level reverse KL and "KL mixing"; read as the convex combination
+     l = (1 - beta) KL(p_t || p_s) + beta KL(p_s || p_t), beta in [0, 1]
+     (beta = 0 is the forward KL of the fused-loss paper).  Undefined for a
+     top-K cache (the student mass outside the support has no teacher value).
 
 Parity pins for every function live in tests/test_oracle_pins.py (closed
 forms, hand-derived fixtures in tests/golden/, library KL routines, autograd,
@@ -163,9 +169,30 @@ def grad_full_rows(s_tilde, lse_s, t_tilde, lse_t, T):
     return (np.exp(s_tilde - lse_s[:, None]) - np.exp(t_tilde - lse_t[:, None])) / T
 
 
+def kl_reverse_rows(s_tilde, lse_s, t_tilde, lse_t):
+    """Per-row reverse KL: l_n = sum_j p_s[j] * (log p_s[j] - log p_t[j])."""
+    log_pt = t_tilde - lse_t[:, None]
+    log_ps = s_tilde - lse_s[:, None]
+    p_s = np.exp(log_ps)
+    return np.sum(p_s * (log_ps - log_pt), axis=1)
+
+
+def grad_reverse_rows(s_tilde, lse_s, t_tilde, lse_t, T):
+    """d l_n / d s (raw logits) for the reverse KL: p_s[j] (u_j - u_bar) / T with
+    u = log p_s - log p_t and u_bar = sum_j p_s[j] u_j.
+    Derivation: d/ds~_k sum_j p_s[j] u_j = sum_j p_s[j] ([j=k] - p_s[k]) u_j
+    + p_s[k] - p_s[k] sum_j p_s[j] = p_s[k] (u_k - u_bar)."""
+    log_ps = s_tilde - lse_s[:, None]
+    u = log_ps - (t_tilde - lse_t[:, None])
+    p_s = np.exp(log_ps)
+    u_bar = np.sum(p_s * u, axis=1, keepdims=True)
+    return p_s * (u - u_bar) / T
+
+
 def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None,
             teacher_lse=None, Ht=None, Wt=None, grad_loss=1.0, normalizer=None,
-            rows=None, vocab_rows=None, want_dH=True, want_dW=True, block=256):
+            rows=None, vocab_rows=None, want_dH=True, want_dW=True, block=256,
+            reverse_weight=0.0):
     """The distillation loss L = (1 / n_valid) * sum_{mask_n = 1} l_n and the
     gradients dH = dS . W, dW = dS^T . H of g * L, with dS = g * dL/ds and g
     the incoming gradient of the loss (readings R1-R5).
@@ -176,6 +203,7 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
     vocab_rows:  rows of dW to return (None = all V).  dW always sums over
                  every token, so it needs all rows' lse.
     normalizer:  divide by this instead of the local unmasked count.
+    reverse_weight: beta of reading R6 (teacher-hidden mode only).
     block:       rows per fp64 matrix product (memory bound only; every row is
                  an independent computation).
 
@@ -187,6 +215,9 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
     V = W.shape[0]
     if T <= 0:
         raise ValueError("temperature must be > 0")
+    beta = float(reverse_weight)
+    if not 0.0 <= beta <= 1.0 or (beta > 0 and mode != HIDDEN):
+        raise ValueError("reverse_weight must be in [0, 1] and needs the teacher-hidden mode")
     keep = np.ones(N, dtype=bool) if mask is None else (_i64(mask) != 0)
     n_valid = int(np.sum(keep))
     norm = float(n_valid if normalizer is None else normalizer)
@@ -215,6 +246,9 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
             lse_t = logsumexp_rows(t)
             l = kl_full_rows(s, lse_s, t, lse_t)
             gr = grad_full_rows(s, lse_s, t, lse_t, T)
+            if beta > 0:
+                l = (1 - beta) * l + beta * kl_reverse_rows(s, lse_s, t, lse_t)
+                gr = (1 - beta) * gr + beta * grad_reverse_rows(s, lse_s, t, lse_t, T)
         k = keep[r]
         l = np.where(k, l, 0.0)
         dS = np.where(k[:, None], coef * gr, 0.0)

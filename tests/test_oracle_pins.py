@@ -64,7 +64,7 @@ def _golden_cases():
 
 @pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
 def test_golden_closed_forms(case):
-    kw = dict(T=case["T"], mode=case["mode"])
+    kw = dict(T=case["T"], mode=case["mode"], reverse_weight=case.get("reverse_weight", 0.0))
     if case.get("mask") is not None:
         kw["mask"] = np.array(case["mask"], dtype=np.uint8)
     if case["mode"] == "topk":
@@ -132,6 +132,37 @@ def test_topk_gradients_match_torch_autograd(partial):
     np.testing.assert_allclose(out["dW"], Wq.grad.numpy(), rtol=1e-10, atol=1e-14)
 
 
+@pytest.mark.parametrize("beta", [1.0, 0.35])
+def test_reverse_and_mixed_kl_match_scipy_and_torch_autograd(beta):
+    H, W, kw = _rand_case(17, N=7, d=5, V=19, mode="hidden", masked=True, T=1.6)
+    out = oracle.kl_loss(H, W, reverse_weight=beta, grad_loss=0.9, **kw)
+    p_s = scipy.special.softmax(H @ W.T / 1.6, axis=1)
+    p_t = scipy.special.softmax(kw["Ht"] @ kw["Wt"].T / 1.6, axis=1)
+    keep = kw["mask"].astype(bool)
+    for n in np.nonzero(keep)[0]:
+        ref = (1 - beta) * scipy.stats.entropy(p_t[n], p_s[n]) + beta * scipy.stats.entropy(
+            p_s[n], p_t[n])
+        assert out["row_loss"][n] == pytest.approx(ref, rel=1e-11, abs=1e-14)
+    Hq = torch.tensor(H, requires_grad=True)
+    Wq = torch.tensor(W, requires_grad=True)
+    log_ps = torch.log_softmax(Hq @ Wq.T / 1.6, dim=1)
+    log_pt = torch.log_softmax(torch.tensor(kw["Ht"]) @ torch.tensor(kw["Wt"]).T / 1.6, dim=1)
+    kl = torch.nn.functional.kl_div
+    rows = ((1 - beta) * kl(log_ps, log_pt, reduction="none", log_target=True).sum(1)
+            + beta * kl(log_pt, log_ps, reduction="none", log_target=True).sum(1))
+    L = rows[torch.tensor(keep)].mean()
+    (0.9 * L).backward()
+    assert out["loss"] == pytest.approx(L.item(), rel=1e-12)
+    np.testing.assert_allclose(out["dH"], Hq.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(out["dW"], Wq.grad.numpy(), rtol=1e-10, atol=1e-14)
+
+
+def test_reverse_weight_needs_teacher_hidden_mode():
+    H, W, kw = _rand_case(18, mode="topk")
+    with pytest.raises(ValueError):
+        oracle.kl_loss(H, W, reverse_weight=0.5, **kw)
+
+
 # ------------------------------------------------------------ finite differences
 
 def _fd_check(H, W, kw, g=1.0, normalizer=None, h=1e-6):
@@ -162,6 +193,13 @@ def _fd_check(H, W, kw, g=1.0, normalizer=None, h=1e-6):
 def test_finite_differences(mode, partial):
     H, W, kw = _rand_case(4, N=5, d=4, V=11, K=3, mode=mode, partial=partial, T=1.7)
     assert _fd_check(H, W, kw, g=0.7) < 1e-7
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.4])
+def test_finite_differences_reverse_and_mixed(beta):
+    H, W, kw = _rand_case(19, N=5, d=4, V=11, mode="hidden", T=1.7)
+    kw = dict(kw, reverse_weight=beta)
+    assert _fd_check(H, W, kw, g=0.8) < 1e-7
 
 
 def test_finite_differences_custom_normalizer():
