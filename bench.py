@@ -46,6 +46,8 @@ def parse():
                     choices=["offline_topk", "full_vocab", "packed_long", "scaling"])
     ap.add_argument("--N", type=int, default=0, help="tokens per GPU (0 = the workload's own)")
     ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--reverse-weight", type=float, default=0.0,
+                    help="teacher-hidden workload: weight of the reverse KL (0 = forward KL)")
     ap.add_argument("--entry", default="fused", choices=["fused", "split"],
                     help="fused: kl_fwd_bwd; split: kl_fwd then kl_bwd (the autograd path, "
                          "backward recomputes the logits)")
@@ -199,6 +201,8 @@ def gpu_arm(args):
     args.N = w.N
     torch.cuda.empty_cache()  # drop the teacher-cache generator's temporaries
     kw = problem_kwargs(w, args.chunk)
+    if args.reverse_weight > 0:
+        kw["reverse_weight"] = args.reverse_weight
     prob, keep = ops.make_problem(w.H, w.W, **kw)
     ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
     loss = torch.empty((), dtype=torch.float32, device=dev)
@@ -276,6 +280,8 @@ def gpu_arm(args):
         devb = {k: torch.empty_like(getattr(w, k)) for k in host}
         hloss = torch.empty((), dtype=torch.float32).pin_memory()
         kw2 = problem_kwargs(w, args.chunk, override=devb)
+        if args.reverse_weight > 0:
+            kw2["reverse_weight"] = args.reverse_weight
         prob2, keep2 = ops.make_problem(devb["H"], w.W, **kw2)
 
         def e2e_step():
@@ -362,6 +368,9 @@ def gpu_arm(args):
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
     if args.workload != "offline_topk":
         line["metric"] = METRIC + f" [{args.workload}]"
+    if args.reverse_weight > 0:
+        line["metric"] += f" [reverse KL weight {args.reverse_weight}]"
+        line["config"]["reverse_weight"] = args.reverse_weight
     if args.entry == "split":
         line["metric"] += " [kl_fwd + kl_bwd]"
         # backward recomputes the student (and teacher) logits once more

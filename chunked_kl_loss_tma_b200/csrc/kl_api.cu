@@ -238,6 +238,9 @@ int validate_shape(const kl_problem* p) {
     return KL_ERR_SHAPE;
   if (!(p->T > 0.f) || !(p->T < INFINITY) || p->chunk_tokens < 0 || !(p->normalizer >= 0.f))
     return KL_ERR_ARG;
+  if (!(p->reverse_weight >= 0.f && p->reverse_weight <= 1.f) ||
+      (p->reverse_weight > 0.f && p->teacher != KL_TEACHER_HIDDEN))
+    return KL_ERR_ARG;
   if (p->d % 8 != 0) return KL_ERR_ALIGN;
   if (p->teacher == KL_TEACHER_TOPK) {
     if (p->K < 1 || p->K > kMaxK) return KL_ERR_SHAPE;
@@ -692,11 +695,12 @@ int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
                         float* row_loss, int write_grad) {
   const kl_problem* p = c.p;
   LaunchScope ls("dlogits_full", c.st, 0,
-                 (write_grad ? 3.0 : 2.0) * Cn * p->V * sizeof(Elem));
+                 ((write_grad ? 3.0 : 2.0) + (p->reverse_weight > 0.f && write_grad ? 2.0 : 0.0)) *
+                     Cn * p->V * sizeof(Elem));
   dlogits_full_kernel<Elem><<<static_cast<unsigned>(Cn), 256, 0, c.st>>>(
       S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
-      row_loss ? row_loss + c0 : nullptr, write_grad);
+      row_loss ? row_loss + c0 : nullptr, write_grad, p->reverse_weight);
   return KL_LAUNCHED();
 }
 

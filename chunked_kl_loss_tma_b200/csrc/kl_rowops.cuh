@@ -301,23 +301,46 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   }
 }
 
-// Full-vocabulary mode (one CTA per row): A = sum_j p_t,j (t~_j - s~_j) so that
-// l = A - lse_t + lse_s; optionally dS = c (p_s - p_t) in place over S.
+// Two block-wide sums in a fixed order (warp shuffles, then warp 0).
+__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
+  a = warp_sum(a);
+  b = warp_sum(b);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(a, b);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float2 v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : make_float2(0.f, 0.f);
+    v.x = warp_sum(v.x);
+    v.y = warp_sum(v.y);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float2 r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// Full-vocabulary mode (one CTA per row).  A = sum_j p_t,j (t~_j - s~_j) gives the
+// forward KL A - lse_t + lse_s; with reverse weight beta > 0 also
+// u_bar = sum_j p_s,j (s~_j - t~_j), the reverse KL u_bar - lse_s + lse_t, and
+//   dS = c [(1 - beta)(p_s - p_t) + beta p_s (u - u_bar)],  u = s~ - t~,
+// written in place over S in a second pass (u_bar is needed first).  With
+// beta = 0 the single pass writes dS = c (p_s - p_t).
 template <typename Elem>
 __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict__ Tt, int64_t ld,
                                     int V, const float* __restrict__ lse_s,
                                     const float* __restrict__ lse_t,
                                     const uint8_t* __restrict__ mask, const Scalars* sc,
                                     const float* g_dev, float g_host, float invT,
-                                    float* __restrict__ row_loss, int write_grad) {
-  __shared__ float red[32];
+                                    float* __restrict__ row_loss, int write_grad, float beta) {
+  __shared__ float2 red[32];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
   const Elem* trow = Tt + static_cast<int64_t>(row) * ld;
   const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT);
   const float ls2 = lse_s[row] * kLog2e, lt2 = lse_t[row] * kLog2e;
   const int nvec = (V + 7) >> 3;
-  float A = 0.f;
+  const bool single = beta == 0.f;
+  float A = 0.f, U = 0.f;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float fs[8], ft[8];
     load8<Elem>(srow + v * 8, fs);
@@ -328,20 +351,35 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
       const float pt = ex2_approx(fmaf(ft[i], kLog2e, -lt2));
       const float ps = ex2_approx(fmaf(fs[i], kLog2e, -ls2));
       A += in ? pt * (ft[i] - fs[i]) : 0.f;
+      U += in ? ps * (fs[i] - ft[i]) : 0.f;
       fs[i] = in ? operand_round<Elem>(coef * (ps - pt)) : 0.f;
     }
-    if (write_grad) store8<Elem>(srow + v * 8, fs);
+    if (write_grad && single) store8<Elem>(srow + v * 8, fs);
   }
-  A = warp_sum(A);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = A;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-    a = warp_sum(a);
-    if (threadIdx.x == 0 && row_loss != nullptr) {
-      const bool keep = mask == nullptr || mask[row] != 0;
-      row_loss[row] = keep ? a - lse_t[row] + lse_s[row] : 0.f;
+  const float2 r = block_sum2(A, U, red);
+  const float ubar = r.y;
+  if (write_grad && !single) {
+    const float cf = coef * (1.f - beta), cr = coef * beta;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float fs[8], ft[8];
+      load8<Elem>(srow + v * 8, fs);
+      load8<Elem>(trow + v * 8, ft);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool in = v * 8 + i < V;
+        const float pt = ex2_approx(fmaf(ft[i], kLog2e, -lt2));
+        const float ps = ex2_approx(fmaf(fs[i], kLog2e, -ls2));
+        const float g = cf * (ps - pt) + cr * ps * ((fs[i] - ft[i]) - ubar);
+        fs[i] = in ? operand_round<Elem>(g) : 0.f;
+      }
+      store8<Elem>(srow + v * 8, fs);
     }
+  }
+  if (threadIdx.x == 0 && row_loss != nullptr) {
+    const bool keep = mask == nullptr || mask[row] != 0;
+    const float fwd = r.x - lse_t[row] + lse_s[row];
+    const float rev = ubar - lse_s[row] + lse_t[row];
+    row_loss[row] = keep ? (1.f - beta) * fwd + beta * rev : 0.f;
   }
 }
 

@@ -38,7 +38,7 @@ def _need(t, name, dtype=None, device=None):
 
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
-                 Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0):
+                 Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0):
     """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive)."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
@@ -60,6 +60,7 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
     p.T = float(T)
     p.chunk_tokens = int(chunk_tokens)
     p.normalizer = float(normalizer)
+    p.reverse_weight = float(reverse_weight)
     keep = [H, W, mask]
     if Ht is not None:
         _need(Ht, "Ht", H.dtype, dev)

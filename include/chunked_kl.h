@@ -19,6 +19,11 @@
  *   KL_TEACHER_HIDDEN (KDFlow abstract: teacher logits recomputed from the
  *       teacher's final hidden states through a frozen teacher head):
  *       t = Ht . Wt^T,  l_n = KL(p_t || p_s),  dl_n/ds_j = (p_s,j - p_t,j) / T.
+ *       With reverse_weight = beta > 0 (the KL-direction study's reverse KL and
+ *       "KL mixing", thelatestinai.com/papers/2606.20005):
+ *       l_n = (1 - beta) KL(p_t || p_s) + beta KL(p_s || p_t),
+ *       dl_n/ds_j = [(1 - beta)(p_s,j - p_t,j) + beta p_s,j (u_j - u_bar)] / T,
+ *       u = s~ - t~, u_bar = sum_j p_s,j u_j.
  *   loss = (1 / n) sum_{mask_n = 1} l_n, n = normalizer if > 0, else the number
  *       of rows with mask = 1 (0 valid rows -> loss 0, gradients 0).
  *   dS = g * dloss/ds (0 on masked rows), dH = dS . W, dW = dS^T . H.
@@ -86,7 +91,8 @@ extern "C" {
 #define KL_ERR_INDEX 7       /* device: cache index outside [-1, V) or duplicated  */
 #define KL_ERR_TIMEOUT 8     /* device: a bounded wait inside a kernel ran out     */
 #define KL_ERR_UNSUPPORTED 9 /* the current device is not sm_100 (B200-class)      */
-#define KL_ERR_ARG 10        /* another bad argument (T <= 0, chunk_tokens < 0...) */
+#define KL_ERR_ARG 10        /* another bad argument (T <= 0, chunk_tokens < 0,
+                                reverse_weight outside [0,1] or set in TOPK mode) */
 #define KL_ERR_TOO_LARGE 11  /* kl_fwd_noalloc: one token row needs more than the
                                 fixed KL_NOALLOC_SCRATCH_BYTES of scratch          */
 
@@ -111,6 +117,8 @@ typedef struct kl_problem {
   int64_t chunk_tokens;      /* token rows per chunk; 0 = library default (4096) */
   float normalizer;          /* > 0: divide by this (e.g. a data-parallel global
                                 count) instead of the number of unmasked rows    */
+  float reverse_weight;      /* HIDDEN: beta in [0, 1], weight of the reverse KL
+                                (0 = forward KL only); must be 0 in TOPK mode    */
 } kl_problem;
 
 /* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if

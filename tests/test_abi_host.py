@@ -70,6 +70,8 @@ def test_workspace_hidden_mode_has_two_logit_buffers(lib):
     ("T", 0.0, 10),           # KL_ERR_ARG
     ("T", -1.0, 10),
     ("chunk_tokens", -5, 10),
+    ("reverse_weight", 0.5, 10),   # reverse KL needs the teacher-hidden mode
+    ("reverse_weight", -0.1, 10),
 ])
 def test_bad_problems_rejected_on_host(lib, field, value, code):
     p = _problem(**{field: value})
@@ -77,6 +79,13 @@ def test_bad_problems_rejected_on_host(lib, field, value, code):
     p.H = p.W = p.topk_idx = p.topk_logit = 256
     rc = L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None)
     assert rc == code, (rc, L.kl_status_string(rc))
+
+
+def test_reverse_weight_range_in_hidden_mode(lib):
+    p = _problem(teacher=1, d_t=4096, K=0, reverse_weight=1.0)
+    assert L.kl_workspace_bytes(p, 2) > 0
+    p.reverse_weight = 1.5
+    assert L.kl_workspace_bytes(p, 2) == 0
 
 
 def test_null_and_misaligned_pointers_rejected(lib):

@@ -47,10 +47,10 @@ def _kw(w):
     return kw
 
 
-def _oracle_rows(w, rows, n_valid, g=1.0):
+def _oracle_rows(w, rows, n_valid, g=1.0, reverse_weight=0.0):
     r = torch.as_tensor(rows, device=w.H.device)
     args = dict(T=w.T, mode=w.mode, grad_loss=g, normalizer=n_valid, want_dW=False,
-                mask=None if w.mask is None else w.mask[r])
+                mask=None if w.mask is None else w.mask[r], reverse_weight=reverse_weight)
     if w.mode == "topk":
         args.update(topk_idx=w.topk_idx[r], topk_logit=w.topk_logit[r],
                     teacher_lse=None if w.teacher_lse is None else w.teacher_lse[r])
@@ -148,6 +148,23 @@ def test_full_vocab_8192_teacher_hidden():
     r = torch.as_tensor(rows, device="cuda")
     np.testing.assert_allclose(f["lse_t"][r].double().cpu().numpy(), ref["lse_t"], rtol=1e-5)
     assert abs(f["loss"].item() - out["loss"].item()) <= 1e-4 * abs(out["loss"].item())
+
+
+def test_full_vocab_8192_mixed_kl():
+    """Forward/reverse mixing (beta = 0.5) at the teacher-hidden configuration."""
+    w = wl.full_vocab(device="cuda", seed=6)
+    kw = dict(_kw(w), reverse_weight=0.5)
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
+    assert ops.status(out["workspace"]) == 0
+    rows = _rows(w.N, None, n_random=12, seed=6)
+    ref = _oracle_rows(w, rows, w.N, reverse_weight=0.5)
+    r = torch.as_tensor(rows, device="cuda")
+    rl = out["row_loss"][r].double().cpu().numpy()
+    assert np.max(np.abs(rl - ref["row_loss"])) <= 2e-3 * np.max(np.abs(ref["row_loss"]))
+    dH = out["dH"][r].double().cpu().numpy()
+    assert np.max(np.abs(dH - ref["dH"])) <= 2e-2 * np.max(np.abs(ref["dH"]))
+    _loss_is_mean_of_rows(out, w.N)
+    _identities(w, out)
 
 
 def test_packed_long_32768_masked():

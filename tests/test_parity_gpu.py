@@ -247,3 +247,23 @@ def test_bitwise_deterministic_across_calls():
     b = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
     for k in ("loss", "row_loss", "dH", "dW"):
         assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.35])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_reverse_and_mixed_kl_fused_and_split(beta, dtype):
+    w = _small_hidden(dtype=dtype, seed=28)
+    kw = dict(_kw(w, chunk=96), reverse_weight=beta)
+    ref = _oracle(w, reverse_weight=beta, grad_loss=1.4)
+    out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=1.4, want_row_loss=True, **kw)
+    _check_loss(out["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(out["row_loss"].cpu().numpy(), ref["row_loss"], rtol=5e-3,
+                               atol=2e-4)
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    _check_loss(f["loss"].item(), ref["loss"])
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"],
+                   grad_loss=torch.full((), 1.4, device="cuda"), **kw)
+    _check_grad(b["dH"], ref["dH"], "dH (split)")
+    _check_grad(b["dW"], ref["dW"], "dW (split)")
