@@ -43,6 +43,11 @@ Readings where the pages are silent (all restated in the design doc):
      l = (1 - beta) KL(p_t || p_s) + beta KL(p_s || p_t), beta in [0, 1]
      (beta = 0 is the forward KL of the fused-loss paper).  Undefined for a
      top-K cache (the student mass outside the support has no teacher value).
+  R7 per-token temperature: the entropy-adaptive KD abstract on page 4
+     (thelatestinai.com/papers/2610.07706) adjusts the distillation temperature
+     per token; read as T given per row (T_n divides row n's student and
+     teacher logits, and its gradient carries 1/T_n).  A scalar T is the same
+     value for every row.
 
 Parity pins for every function live in tests/test_oracle_pins.py (closed
 forms, hand-derived fixtures in tests/golden/, library KL routines, autograd,
@@ -91,11 +96,18 @@ def logsumexp_rows(x):
     return (m + np.log(np.sum(np.exp(x - m), axis=1, keepdims=True)))[:, 0]
 
 
+def _col(T):
+    """Temperature as a column to divide row blocks by (scalar or one per row)."""
+    T = np.asarray(T, dtype=np.float64)
+    return T if T.ndim == 0 else T[:, None]
+
+
 def scaled_logits(X, Wh, T):
     """x~ = (X . Wh^T) / T for a block of rows: the output projection of the
     head (§3 "Fused chunked KL": the loss integrates the output projection)
-    followed by temperature scaling (reading R1).  fp64 matrix product."""
-    return (X @ Wh.T) / T
+    followed by temperature scaling (readings R1, R7: T scalar or one per
+    row).  fp64 matrix product."""
+    return (X @ Wh.T) / _col(T)
 
 
 def teacher_support_probs(topk_idx, topk_logit, T, teacher_lse, V):
@@ -109,7 +121,7 @@ def teacher_support_probs(topk_idx, topk_logit, T, teacher_lse, V):
         entries of t/T.
     Empty slots (index -1) get q = 0 (reading R4)."""
     idx = _i64(topk_idx)
-    t = _f64(topk_logit) / T
+    t = _f64(topk_logit) / _col(T)
     valid = idx >= 0
     if np.any(idx >= V) or np.any(idx < -1):
         raise ValueError("top-K index out of range")
@@ -151,7 +163,7 @@ def grad_topk_rows(s_tilde, lse_s, idx, q, valid, T):
     for i in range(idx.shape[1]):
         sel = valid[:, i]
         g[rows[sel], idx[sel, i]] -= q[sel, i]
-    return g / T
+    return g / _col(T)
 
 
 def kl_full_rows(s_tilde, lse_s, t_tilde, lse_t):
@@ -166,7 +178,7 @@ def kl_full_rows(s_tilde, lse_s, t_tilde, lse_t):
 
 def grad_full_rows(s_tilde, lse_s, t_tilde, lse_t, T):
     """d l_n / d s (raw logits) for the full KL: (p_s[j] - p_t[j]) / T."""
-    return (np.exp(s_tilde - lse_s[:, None]) - np.exp(t_tilde - lse_t[:, None])) / T
+    return (np.exp(s_tilde - lse_s[:, None]) - np.exp(t_tilde - lse_t[:, None])) / _col(T)
 
 
 def kl_reverse_rows(s_tilde, lse_s, t_tilde, lse_t):
@@ -186,7 +198,7 @@ def grad_reverse_rows(s_tilde, lse_s, t_tilde, lse_t, T):
     u = log_ps - (t_tilde - lse_t[:, None])
     p_s = np.exp(log_ps)
     u_bar = np.sum(p_s * u, axis=1, keepdims=True)
-    return p_s * (u - u_bar) / T
+    return p_s * (u - u_bar) / _col(T)
 
 
 def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None,
@@ -204,6 +216,7 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
                  every token, so it needs all rows' lse.
     normalizer:  divide by this instead of the local unmasked count.
     reverse_weight: beta of reading R6 (teacher-hidden mode only).
+    T:           scalar, or one temperature per token row (reading R7).
     block:       rows per fp64 matrix product (memory bound only; every row is
                  an independent computation).
 
@@ -213,8 +226,9 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
     W = _f64(W)
     N, d = H.shape
     V = W.shape[0]
-    if T <= 0:
-        raise ValueError("temperature must be > 0")
+    T_all = _f64(T)
+    if np.any(T_all <= 0) or (T_all.ndim == 1 and T_all.shape[0] != N) or T_all.ndim > 1:
+        raise ValueError("temperature must be > 0 (scalar or one per row)")
     beta = float(reverse_weight)
     if not 0.0 <= beta <= 1.0 or (beta > 0 and mode != HIDDEN):
         raise ValueError("reverse_weight must be in [0, 1] and needs the teacher-hidden mode")
@@ -223,8 +237,11 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
     norm = float(n_valid if normalizer is None else normalizer)
     coef = (grad_loss / norm) if norm > 0 else 0.0
 
+    def T_of(r):
+        return T_all if T_all.ndim == 0 else T_all[r]
+
     if mode == TOPK:
-        idx_all, q_all, valid_all = teacher_support_probs(topk_idx, topk_logit, T,
+        idx_all, q_all, valid_all = teacher_support_probs(topk_idx, topk_logit, T_all,
                                                           teacher_lse, V)
     elif mode == HIDDEN:
         Ht = _f64(Ht)
@@ -235,20 +252,21 @@ def kl_loss(H, W, *, T=1.0, mask=None, mode=TOPK, topk_idx=None, topk_logit=None
     def block_terms(r):
         """Row losses, lse and dS (= coef * dl/ds, zero on masked rows) for
         the token rows r."""
-        s = scaled_logits(H[r], W, T)
+        Tr = T_of(r)
+        s = scaled_logits(H[r], W, Tr)
         lse_s = logsumexp_rows(s)
         if mode == TOPK:
             l = kl_topk_rows(s, lse_s, idx_all[r], q_all[r], valid_all[r])
-            gr = grad_topk_rows(s, lse_s, idx_all[r], q_all[r], valid_all[r], T)
+            gr = grad_topk_rows(s, lse_s, idx_all[r], q_all[r], valid_all[r], Tr)
             lse_t = None
         else:
-            t = scaled_logits(Ht[r], Wt, T)
+            t = scaled_logits(Ht[r], Wt, Tr)
             lse_t = logsumexp_rows(t)
             l = kl_full_rows(s, lse_s, t, lse_t)
-            gr = grad_full_rows(s, lse_s, t, lse_t, T)
+            gr = grad_full_rows(s, lse_s, t, lse_t, Tr)
             if beta > 0:
                 l = (1 - beta) * l + beta * kl_reverse_rows(s, lse_s, t, lse_t)
-                gr = (1 - beta) * gr + beta * grad_reverse_rows(s, lse_s, t, lse_t, T)
+                gr = (1 - beta) * gr + beta * grad_reverse_rows(s, lse_s, t, lse_t, Tr)
         k = keep[r]
         l = np.where(k, l, 0.0)
         dS = np.where(k[:, None], coef * gr, 0.0)

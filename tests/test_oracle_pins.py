@@ -202,6 +202,33 @@ def test_finite_differences_reverse_and_mixed(beta):
     assert _fd_check(H, W, kw, g=0.8) < 1e-7
 
 
+@pytest.mark.parametrize("mode,partial", [("topk", True), ("topk", False), ("hidden", True)])
+def test_finite_differences_per_token_temperature(mode, partial):
+    H, W, kw = _rand_case(20, N=5, d=4, V=11, K=3, mode=mode, partial=partial)
+    Tr = np.array([0.7, 1.3, 2.1, 1.0, 0.9])
+    kw = dict(kw, T=Tr)
+    if mode == "topk" and partial:  # the cache's lse at each row's own temperature
+        rng = np.random.default_rng(20)
+        kw["teacher_lse"] = kw["teacher_lse"] + rng.normal(scale=0.1, size=5)
+    assert _fd_check(H, W, kw, g=1.1) < 1e-7
+
+
+def test_per_token_temperature_equals_rows_at_their_own_scalar_T():
+    H, W, kw = _rand_case(21, N=6, d=4, V=13, K=4, mode="topk", masked=False)
+    Tr = np.array([0.5, 1.0, 1.5, 2.0, 2.5, 3.0])
+    t = kw["topk_logit"]
+    both = oracle.kl_loss(H, W, **dict(kw, T=Tr))
+    dW = np.zeros_like(W)
+    for n in range(6):
+        one = oracle.kl_loss(H[n:n + 1], W, T=float(Tr[n]), mode="topk",
+                             topk_idx=kw["topk_idx"][n:n + 1], topk_logit=t[n:n + 1],
+                             teacher_lse=kw["teacher_lse"][n:n + 1], normalizer=6)
+        assert both["row_loss"][n] == pytest.approx(one["row_loss"][0], rel=1e-13)
+        np.testing.assert_allclose(both["dH"][n], one["dH"][0], rtol=1e-12, atol=1e-16)
+        dW += one["dW"]
+    np.testing.assert_allclose(both["dW"], dW, rtol=1e-11, atol=1e-16)
+
+
 def test_finite_differences_custom_normalizer():
     H, W, kw = _rand_case(5, N=4, d=3, V=9, K=3, mode="topk", T=0.9)
     assert _fd_check(H, W, kw, g=1.3, normalizer=11.0) < 1e-7
