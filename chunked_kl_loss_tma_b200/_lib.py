@@ -41,7 +41,7 @@ class KLProblem(ctypes.Structure):
         ("teacher_lse", ctypes.c_void_p),
         ("d_t", ctypes.c_int64), ("Ht", ctypes.c_void_p), ("Wt", ctypes.c_void_p),
         ("chunk_tokens", ctypes.c_int64), ("normalizer", ctypes.c_float),
-        ("reverse_weight", ctypes.c_float),
+        ("reverse_weight", ctypes.c_float), ("T_row", ctypes.c_void_p),
     ]
 
 

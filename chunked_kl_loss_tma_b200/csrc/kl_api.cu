@@ -433,6 +433,7 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
   gp.scale = c.invT;
+  gp.T_row = p->T_row ? p->T_row + c0 : nullptr;
   gp.partials = partials;
   gp.sidx = sidx;
   gp.sq = sq;
@@ -531,6 +532,7 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
   gp.scale = c.invT;
+  gp.T_row = p->T_row ? p->T_row + c0 : nullptr;
   gp.sidx = reinterpret_cast<const int*>(c.ws + c.pl.off_sidx);
   gp.sq = reinterpret_cast<const float*>(c.ws + c.pl.off_sq);
   gp.ktop = p->K;
@@ -627,7 +629,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
 
 int launch_count_valid(Ctx& c) {
   LaunchScope ls("count_valid", c.st, 0, static_cast<double>(c.p->mask ? c.p->N : 0));
-  count_valid_kernel<<<1, 1024, 0, c.st>>>(c.p->mask, c.p->N, c.p->normalizer, c.sc);
+  count_valid_kernel<<<1, 1024, 0, c.st>>>(c.p->mask, c.p->N, c.p->normalizer, c.p->T_row, c.sc);
   return KL_LAUNCHED();
 }
 
@@ -651,6 +653,7 @@ int launch_prep(Ctx& c, int64_t c0, int64_t Cn) {
   prep_topk_kernel<<<static_cast<unsigned>(cdiv(Cn, rows_per_block)), 32 * rows_per_block, smem,
                      c.st>>>(p->topk_idx + c0 * K, p->topk_logit + c0 * K,
                              p->teacher_lse ? p->teacher_lse + c0 : nullptr, c.invT,
+                             p->T_row ? p->T_row + c0 : nullptr,
                              static_cast<int>(p->V), K, static_cast<int>(Cn), sidx, sq, rinfo,
                              c.sc);
   return KL_LAUNCHED();
@@ -685,7 +688,8 @@ int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* ls
       S, c.pl.Vp, static_cast<int>(p->V), lse + c0, p->mask ? p->mask + c0 : nullptr,
       reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
       reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
-      reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT);
+      reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT,
+      p->T_row ? p->T_row + c0 : nullptr);
   return KL_LAUNCHED();
 }
 
@@ -700,7 +704,8 @@ int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
   dlogits_full_kernel<Elem><<<static_cast<unsigned>(Cn), 256, 0, c.st>>>(
       S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
-      row_loss ? row_loss + c0 : nullptr, write_grad, p->reverse_weight);
+      p->T_row ? p->T_row + c0 : nullptr, row_loss ? row_loss + c0 : nullptr, write_grad,
+      p->reverse_weight);
   return KL_LAUNCHED();
 }
 

@@ -81,7 +81,8 @@ struct GemmParams {
   int store;           // STATS: store s~ through the output map (0 = statistics only)
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
-  float scale;         // STATS: 1 / T
+  float scale;         // STATS / DLOGITS: 1 / T
+  const float* T_row;  // STATS / DLOGITS: per-row temperature (chunk rows), or nullptr
   int beta;            // ACCUM: 0 overwrite, 1 accumulate
   float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross, 0)
   const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
@@ -451,7 +452,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int col0 = tn * kBN;
 
       if (EPI == EPI_STATS) {
-        const float s2 = p.scale * kLog2e;
+        const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
+        const float s2 = rscale * kLog2e;
         float mx = -INFINITY, se = 0.f, cross = 0.f;
         int gi = 0, gcol = 0x7fffffff;
         const int* ri = nullptr;
@@ -498,17 +500,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float val = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) val = (i == k) ? __uint_as_float(v[i]) : val;
-            cross += __ldg(rq + gi) * (val * p.scale);
+            cross += __ldg(rq + gi) * (val * rscale);
             ++gi;
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
           if (p.store && cb < p.cols_valid)
-            store_box(v, p.scale, cb, row0, kElemF32, false, warp_rows);
+            store_box(v, rscale, cb, row0, kElemF32, false, warp_rows);
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
       } else if (EPI == EPI_DLOGITS) {
         float coef = 0.f, cm = 0.f, l2 = 0.f;
+        const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
         int gi = 0, gcol = 0x7fffffff;
         const int* ri = nullptr;
         const float* rq = nullptr;
@@ -516,7 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const bool keep = p.mask == nullptr || p.mask[grow] != 0;
           const float g = p.g_dev != nullptr ? *p.g_dev : p.g_host;
           const float n = *p.norm;
-          coef = (keep && n > 0.f) ? g / n * p.scale : 0.f;
+          coef = (keep && n > 0.f) ? g / n * rscale : 0.f;
           cm = coef * p.rowinfo[grow].x;
           l2 = p.lse[grow] * kLog2e;
           ri = p.sidx + static_cast<int64_t>(grow) * p.ktop;
@@ -529,7 +532,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
-        const float s2 = p.scale * kLog2e;
+        const float s2 = rscale * kLog2e;
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t v[32];

@@ -15,6 +15,12 @@
 namespace ckl {
 
 constexpr int kStatusIndex = 7;  // KL_ERR_INDEX
+constexpr int kStatusArg = 10;   // KL_ERR_ARG (a per-token temperature <= 0)
+
+// 1 / T for a row: the row's own temperature when T_row is given.
+__device__ __forceinline__ float row_invT(const float* T_row, int row, float invT) {
+  return T_row != nullptr ? 1.f / T_row[row] : invT;
+}
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kEmpty = 0x7fffffff;  // sorted-cache sentinel for an empty slot
 
@@ -118,10 +124,16 @@ __device__ __forceinline__ void store8<float>(float* dst, const float* f) {
 
 // Resets the status word and counts the rows that enter the mean.
 __global__ void count_valid_kernel(const uint8_t* mask, int64_t N, float normalizer,
-                                   Scalars* sc) {
+                                   const float* T_row, Scalars* sc) {
   __shared__ int part[32];
+  __shared__ int badT;
+  if (threadIdx.x == 0) badT = 0;
+  __syncthreads();
   int c = 0;
-  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) c += mask ? (mask[i] != 0) : 1;
+  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) {
+    c += mask ? (mask[i] != 0) : 1;
+    if (T_row != nullptr && !(T_row[i] > 0.f)) badT = 1;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
@@ -129,7 +141,7 @@ __global__ void count_valid_kernel(const uint8_t* mask, int64_t N, float normali
   if (threadIdx.x == 0) {
     int tot = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
-    sc->status = 0;
+    sc->status = badT ? kStatusArg : 0;
     sc->n_valid = tot;
     sc->norm = normalizer > 0.f ? normalizer : static_cast<float>(tot);
   }
@@ -143,8 +155,9 @@ __global__ void count_valid_kernel(const uint8_t* mask, int64_t N, float normali
 // rowinfo = (m = sum q, sum q log q).
 __global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
                                  const float* __restrict__ logit,
-                                 const float* __restrict__ lse_t, float invT, int V, int K,
-                                 int rows, int* __restrict__ sidx, float* __restrict__ sq,
+                                 const float* __restrict__ lse_t, float invT,
+                                 const float* __restrict__ T_row, int V, int K, int rows,
+                                 int* __restrict__ sidx, float* __restrict__ sq,
                                  float2* __restrict__ rowinfo, Scalars* sc) {
   extern __shared__ int prep_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -157,6 +170,7 @@ __global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
   const float* rl = logit + static_cast<int64_t>(row) * K;
   bool bad = false;
   float tmax = -INFINITY;
+  invT = row_invT(T_row, row, invT);
   for (int i = lane; i < K; i += 32) {
     int k = ri[i];
     if (k < -1 || k >= V) {
@@ -246,7 +260,9 @@ __global__ void row_reduce_kernel(const float4* __restrict__ partials, int tiles
 }
 
 __device__ __forceinline__ float grad_coef(const uint8_t* mask, int row, const Scalars* sc,
-                                           const float* g_dev, float g_host, float invT) {
+                                           const float* g_dev, float g_host, float invT,
+                                           const float* T_row) {
+  invT = row_invT(T_row, row, invT);
   const bool keep = mask == nullptr || mask[row] != 0;
   const float g = g_dev != nullptr ? *g_dev : g_host;
   const float norm = sc->norm;
@@ -262,11 +278,11 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
                                     const float2* __restrict__ rowinfo,
                                     const int* __restrict__ sidx, const float* __restrict__ sq,
                                     int K, const Scalars* sc, const float* g_dev, float g_host,
-                                    float invT) {
+                                    float invT, const float* __restrict__ T_row) {
   extern __shared__ float sval[];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
-  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT);
+  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
   const int nvec = (V + 7) >> 3;
   if (coef == 0.f) {
     const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -331,12 +347,13 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
                                     const float* __restrict__ lse_t,
                                     const uint8_t* __restrict__ mask, const Scalars* sc,
                                     const float* g_dev, float g_host, float invT,
+                                    const float* __restrict__ T_row,
                                     float* __restrict__ row_loss, int write_grad, float beta) {
   __shared__ float2 red[32];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
   const Elem* trow = Tt + static_cast<int64_t>(row) * ld;
-  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT);
+  const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
   const float ls2 = lse_s[row] * kLog2e, lt2 = lse_t[row] * kLog2e;
   const int nvec = (V + 7) >> 3;
   const bool single = beta == 0.f;

@@ -39,6 +39,7 @@ def _need(t, name, dtype=None, device=None):
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
                  Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0):
+    """T: a number, or a float32 tensor [N] of per-token temperatures."""
     """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive)."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
@@ -57,11 +58,18 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
     p.V = W.shape[0]
     p.dtype = _DT[H.dtype]
     p.H, p.W, p.mask = _ptr(H), _ptr(W), _ptr(mask)
+    T_row = None
+    if isinstance(T, torch.Tensor):
+        T_row = _need(T, "T", torch.float32, dev)
+        if T_row.shape != (H.shape[0],):
+            raise ValueError("a per-token T must be [N]")
+        T = 1.0
     p.T = float(T)
+    p.T_row = _ptr(T_row)
     p.chunk_tokens = int(chunk_tokens)
     p.normalizer = float(normalizer)
     p.reverse_weight = float(reverse_weight)
-    keep = [H, W, mask]
+    keep = [H, W, mask, T_row]
     if Ht is not None:
         _need(Ht, "Ht", H.dtype, dev)
         _need(Wt, "Wt", H.dtype, dev)

@@ -40,7 +40,7 @@ class Workload:
     N: int
     d: int
     V: int
-    T: float
+    T: "float | torch.Tensor"                    # scalar, or float32 [N] per token
     mode: str
     dtype: torch.dtype
     H: torch.Tensor
@@ -57,9 +57,9 @@ class Workload:
 
     def to(self, device):
         kw = {}
-        for k in ("H", "W", "mask", "topk_idx", "topk_logit", "teacher_lse", "Ht", "Wt"):
+        for k in ("H", "W", "mask", "topk_idx", "topk_logit", "teacher_lse", "Ht", "Wt", "T"):
             v = getattr(self, k)
-            kw[k] = None if v is None else v.to(device)
+            kw[k] = v.to(device) if isinstance(v, torch.Tensor) else v
         return Workload(**{**self.__dict__, **kw})
 
 
@@ -79,7 +79,8 @@ def _normal(shape, std, dtype, g, device):
 def teacher_topk_cache(Ht, Wt, K, T, rows_per_block=2048):
     """Teacher cache for rows of Ht: the K largest logits of Ht . Wt^T (fp32
     products of the stored values, descending), their int32 indices, and the
-    full-vocabulary log-sum-exp of logits / T."""
+    full-vocabulary log-sum-exp of logits / T (T a number, or a tensor with one
+    temperature per row)."""
     N = Ht.shape[0]
     idx = torch.empty(N, K, dtype=torch.int32, device=Ht.device)
     val = torch.empty(N, K, dtype=torch.float32, device=Ht.device)
@@ -93,7 +94,9 @@ def teacher_topk_cache(Ht, Wt, K, T, rows_per_block=2048):
             v, i = torch.topk(t, K, dim=1, largest=True, sorted=True)
             idx[b:b + rows_per_block] = i.to(torch.int32)
             val[b:b + rows_per_block] = v
-            lse[b:b + rows_per_block] = torch.logsumexp(t.double() / T, dim=1).float()
+            Tb = T[b:b + rows_per_block].to(t.device).double()[:, None] \
+                if isinstance(T, torch.Tensor) else T
+            lse[b:b + rows_per_block] = torch.logsumexp(t.double() / Tb, dim=1).float()
             del t
     finally:
         torch.backends.cuda.matmul.allow_tf32 = prev
@@ -102,7 +105,8 @@ def teacher_topk_cache(Ht, Wt, K, T, rows_per_block=2048):
 
 def make_topk(name, N, d, V, K, d_t, T, dtype, w_std, tw_std, seed, device="cpu",
               mask=None, partial_mass=True, meta=None):
-    """Student H, W and a teacher top-K cache from a separate random teacher."""
+    """Student H, W and a teacher top-K cache from a separate random teacher.
+    T may be a float32 tensor [N] of per-token temperatures."""
     g = _gen(seed, device)
     H = _normal((N, d), 1.0, dtype, g, device)
     W = _normal((V, d), w_std, dtype, g, device)

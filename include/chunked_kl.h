@@ -119,6 +119,13 @@ typedef struct kl_problem {
                                 count) instead of the number of unmasked rows    */
   float reverse_weight;      /* HIDDEN: beta in [0, 1], weight of the reverse KL
                                 (0 = forward KL only); must be 0 in TOPK mode    */
+  const float* T_row;        /* [N] device: temperature per token row (each > 0),
+                                overriding T (the entropy-adaptive KD abstract,
+                                thelatestinai.com/papers/2610.07706, adjusts the
+                                temperature per token); NULL = T for every row.
+                                teacher_lse must then be taken at each row's T.
+                                A value <= 0 is flagged as KL_ERR_ARG in the
+                                device status (kl_status).                       */
 } kl_problem;
 
 /* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if

@@ -267,3 +267,51 @@ def test_reverse_and_mixed_kl_fused_and_split(beta, dtype):
                    grad_loss=torch.full((), 1.4, device="cuda"), **kw)
     _check_grad(b["dH"], ref["dH"], "dH (split)")
     _check_grad(b["dW"], ref["dW"], "dW (split)")
+
+
+def _per_token_T(N, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (0.5 + 2.0 * torch.rand(N, generator=g)).float()
+
+
+@pytest.mark.parametrize("partial", [True, False])
+def test_per_token_temperature_topk_fused_and_split(partial):
+    Tr = _per_token_T(300, 29)
+    w = wl.make_topk("ptt", N=300, d=200, V=5003, K=16, d_t=64, T=Tr, dtype=torch.bfloat16,
+                     w_std=0.05, tw_std=0.1, seed=29, partial_mass=partial).to("cuda")
+    w.mask = torch.ones(300, dtype=torch.uint8, device="cuda")
+    w.mask[::6] = 0
+    kw = _kw(w, chunk=128)
+    ref = _oracle(w, grad_loss=0.8)
+    out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=0.8, want_row_loss=True, **kw)
+    assert ops.status(out["workspace"]) == 0
+    _check_loss(out["loss"].item(), ref["loss"])
+    np.testing.assert_allclose(out["row_loss"].cpu().numpy(), ref["row_loss"], rtol=5e-3,
+                               atol=2e-4)
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], grad_loss=torch.full((), 0.8, device="cuda"), **kw)
+    _check_loss(f["loss"].item(), ref["loss"])
+    _check_grad(b["dH"], ref["dH"], "dH (split)")
+    _check_grad(b["dW"], ref["dW"], "dW (split)")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_per_token_temperature_hidden_mixed(dtype):
+    w = _small_hidden(dtype=dtype, seed=30)
+    w.T = _per_token_T(w.N, 30).to("cuda")
+    kw = dict(_kw(w, chunk=96), reverse_weight=0.25)
+    ref = _oracle(w, reverse_weight=0.25)
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_non_positive_per_token_temperature_sets_status():
+    w = _small_topk(seed=31)
+    Tr = torch.ones(w.N, device="cuda")
+    Tr[17] = 0.0
+    out = ops.kl_fwd_bwd(w.H, w.W, **dict(_kw(w), T=Tr))
+    assert ops.status(out["workspace"]) == 10  # KL_ERR_ARG
