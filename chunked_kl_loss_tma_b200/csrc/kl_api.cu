@@ -21,6 +21,7 @@
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <deque>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -120,7 +121,7 @@ struct ProfKind {
 };
 std::mutex g_prof_mu;
 bool g_prof_on = false;
-std::vector<ProfKind> g_prof;
+std::deque<ProfKind> g_prof;  // deque: LaunchScope keeps pointers to its entries
 std::vector<cudaEvent_t> g_ev_pool;
 
 cudaEvent_t pool_event() {
@@ -330,14 +331,14 @@ template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
   auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR>;
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load()) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
         cudaSuccess)
       return KL_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true);
   }
   const int tiles = gp.tiles_m * gp.tiles_n * gp.ksplit;  // work units
   const int units = PAIR ? sms / 2 : sms;  // CTA pairs or CTAs, one CTA per SM
@@ -641,13 +642,13 @@ int launch_prep(Ctx& c, int64_t c0, int64_t Cn) {
   int* sidx = reinterpret_cast<int*>(c.ws + c.pl.off_sidx);
   float* sq = reinterpret_cast<float*>(c.ws + c.pl.off_sq);
   float2* rinfo = reinterpret_cast<float2*>(c.ws + c.pl.off_rinfo);
-  static bool attr[kMaxDevices] = {};
+  static std::atomic<bool> attr[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr[dev]) {
+  if (!attr[dev].load()) {
     cudaFuncSetAttribute(prep_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          rows_per_block * 3 * kMaxK * 4);
-    attr[dev] = true;
+    attr[dev].store(true);
   }
   LaunchScope ls("prep_topk", c.st, 0, static_cast<double>(Cn) * K * 16 + Cn * 12);
   prep_topk_kernel<<<static_cast<unsigned>(cdiv(Cn, rows_per_block)), 32 * rows_per_block, smem,
@@ -675,13 +676,13 @@ template <typename Elem>
 int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse,
                         const float* g_dev, float g_host) {
   const kl_problem* p = c.p;
-  static bool attr[kMaxDevices] = {};
+  static std::atomic<bool> attr[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr[dev]) {
+  if (!attr[dev].load()) {
     cudaFuncSetAttribute(dlogits_topk_kernel<Elem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kMaxK * 4);
-    attr[dev] = true;
+    attr[dev].store(true);
   }
   LaunchScope ls("dlogits_topk", c.st, 0, 2.0 * Cn * p->V * sizeof(Elem));
   dlogits_topk_kernel<Elem><<<static_cast<unsigned>(Cn), 256, p->K * 4, c.st>>>(
@@ -776,10 +777,10 @@ template <typename Elem>
 int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
             void* dH, float* dW, int accumulate) {
   const kl_problem* p = c.p;
+  KL_TRY(launch_count_valid(c));  // also resets the status word
   if (p->N == 0) return accumulate ? KL_OK : launch_fill(c, dW, p->V * p->d, 0.f);
   Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
   Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
-  KL_TRY(launch_count_valid(c));
   KL_TRY(prepare_heads(c));
   if (sizeof(Elem) == 4)
     KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
@@ -933,7 +934,6 @@ int kl_profile_begin(void) {
       g_ev_pool.push_back(e.second);
     }
   g_prof.clear();
-  g_prof.reserve(64);
   g_prof_on = true;
   return KL_OK;
 }

@@ -39,9 +39,9 @@
  *   - Row-major layouts.  H [N, d], W [V, d], Ht [N, d_t], Wt [V, d_t],
  *     topk_idx/topk_logit [N, K], mask/teacher_lse/lse/row_loss [N],
  *     dH [N, d] (same dtype as H), dW [V, d] float32.
- *   - Alignment: H, W, Ht, Wt, dH, dW and the workspace must be 16-byte
- *     aligned, and d, d_t must make rows a multiple of 16 bytes
- *     (multiple of 8 for bf16, of 4 for fp32).  Violations return KL_ERR_ALIGN.
+ *   - Alignment: H, W, Ht, Wt, dH, dW must be 16-byte aligned, the workspace
+ *     256-byte aligned, and d, d_t multiples of 8 (for both element types).
+ *     Violations return KL_ERR_ALIGN.
  *   - stream is a cudaStream_t (passed as void*; NULL = legacy default
  *     stream).  Calls are asynchronous on it; no host synchronisation happens
  *     inside a call.  Host-detectable errors (NULL, shape, dtype, alignment,
