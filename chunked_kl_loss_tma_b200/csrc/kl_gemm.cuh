@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = warp * 32 + lane;  // accumulator row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     uint8_t* stg = staging + warp * 2 * kStageOutBytes;
+    const uint64_t out_policy = l2_policy_evict_first();
     uint32_t nbox = 0;  // output boxes this warp has staged
     uint32_t local = 0;
     // The accumulator stage is released with one arrival per warp on the
@@ -429,8 +430,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && issue) {
-        if (reduce) tma_reduce_add_2d(&tmC, sb, x, y);
-        else tma_store_2d(&tmC, sb, x, y);
+        // outputs are streamed, never re-read by this kernel: evict them from
+        // L2 first so the operand tiles that other tiles share stay resident
+        if (reduce) tma_reduce_add_2d_hint(&tmC, sb, x, y, out_policy);
+        else tma_store_2d_hint(&tmC, sb, x, y, out_policy);
         bulk_commit();
       }
     };
