@@ -91,6 +91,12 @@ def problem_kwargs(w, chunk, override=None):
     return kw
 
 
+def _pg_timeout():
+    import datetime
+
+    return datetime.timedelta(seconds=int(os.environ.get("KL_BENCH_PG_TIMEOUT", "600")))
+
+
 def dist_setup(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -193,10 +199,17 @@ def gpu_arm(args):
     from chunked_kl_loss_tma_b200.dist import max_over_ranks
 
     ws, rank, local = dist_setup(args)
+    local = local % max(torch.cuda.device_count(), 1)  # ranks beyond the devices share them
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if ws > 1:
-        dist.init_process_group("nccl", device_id=dev)
+        # KL_BENCH_BACKEND=gloo runs the same multi-rank path with host-side
+        # collectives (e.g. several ranks sharing one GPU for a functional check)
+        backend = os.environ.get("KL_BENCH_BACKEND", "nccl")
+        if backend == "nccl":
+            dist.init_process_group("nccl", device_id=dev, timeout=_pg_timeout())
+        else:
+            dist.init_process_group(backend, timeout=_pg_timeout())
     w = make_workload(wl, args, dev, rank)
     args.N = w.N
     torch.cuda.empty_cache()  # drop the teacher-cache generator's temporaries
