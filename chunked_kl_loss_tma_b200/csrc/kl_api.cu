@@ -674,7 +674,7 @@ int launch_row_reduce(Ctx& c, const float4* partials, int64_t c0, int64_t Cn, bo
 
 template <typename Elem>
 int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse,
-                        const float* g_dev, float g_host) {
+                        const float* g_dev, float g_host, const float4* part) {
   const kl_problem* p = c.p;
   static std::atomic<bool> attr[kMaxDevices];
   int dev = 0;
@@ -690,14 +690,15 @@ int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* ls
       reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
       reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
       reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT,
-      p->T_row ? p->T_row + c0 : nullptr);
+      p->T_row ? p->T_row + c0 : nullptr, part, c.pl.tiles_v);
   return KL_LAUNCHED();
 }
 
 template <typename Elem>
 int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
                         const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
-                        float* row_loss, int write_grad) {
+                        float* row_loss, int write_grad, const float4* part_s,
+                        const float4* part_t) {
   const kl_problem* p = c.p;
   LaunchScope ls("dlogits_full", c.st, 0,
                  ((write_grad ? 3.0 : 2.0) + (p->reverse_weight > 0.f && write_grad ? 2.0 : 0.0)) *
@@ -706,7 +707,7 @@ int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
       S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
       p->T_row ? p->T_row + c0 : nullptr, row_loss ? row_loss + c0 : nullptr, write_grad,
-      p->reverse_weight);
+      p->reverse_weight, part_s, part_t, c.pl.tiles_v);
   return KL_LAUNCHED();
 }
 
@@ -767,7 +768,8 @@ int run_fwd(Ctx& c, float* loss, float* lse_s, float* lse_t, float* row_loss) {
                                "gemm_teacher_logits"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
       KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, 0.f, rl, 0));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, 0.f, rl, 0, ps,
+                                       pt));
     }
   }
   return launch_finalize(c, rl, loss);
@@ -795,8 +797,9 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
                                "gemm_logits_recompute"));
       KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, nullptr, nullptr, nullptr,
                                0, "gemm_teacher_logits"));
+      // backward: logits were recomputed without tile statistics (not shifted)
       KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, g_dev, g_host, nullptr,
-                                       1));
+                                       1, nullptr, nullptr));
     }
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
   }
@@ -832,7 +835,7 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                                "gemm_logits_stats"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
-      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g));
+      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
     } else {
       KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
                                "gemm_logits_stats"));
@@ -840,7 +843,7 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
                                "gemm_teacher_logits"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
       KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1, ps, pt));
     }
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
   }

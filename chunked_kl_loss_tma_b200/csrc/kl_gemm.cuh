@@ -401,8 +401,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     };
     // Stage v * scale (32 values of this thread's row) and store the warp's box
     // at output column x, output-map row y (rows past row_end are not written).
-    auto store_box = [&](const uint32_t(&v)[32], float scale, int x, int y, bool fp32_out,
-                         bool reduce, bool issue) {
+    // (stores v * scale - shift)
+    auto store_box = [&](const uint32_t(&v)[32], float scale, float shift, int x, int y,
+                         bool fp32_out, bool reduce, bool issue) {
       uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
       ++nbox;
       if (lane == 0) bulk_wait_read_1();  // the store that last used sb has read it
@@ -410,10 +411,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (fp32_out) {  // 128-byte rows, 128-byte swizzle: chunk j at j ^ (row & 7)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 q = make_float4(__uint_as_float(v[4 * j]) * scale,
-                                       __uint_as_float(v[4 * j + 1]) * scale,
-                                       __uint_as_float(v[4 * j + 2]) * scale,
-                                       __uint_as_float(v[4 * j + 3]) * scale);
+          const float4 q = make_float4(fmaf(__uint_as_float(v[4 * j]), scale, -shift),
+                                       fmaf(__uint_as_float(v[4 * j + 1]), scale, -shift),
+                                       fmaf(__uint_as_float(v[4 * j + 2]), scale, -shift),
+                                       fmaf(__uint_as_float(v[4 * j + 3]), scale, -shift));
           *reinterpret_cast<float4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) = q;
         }
       } else {  // bf16: 64-byte rows, 64-byte swizzle: chunk j at j ^ ((row >> 1) & 3)
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int j = 0; j < 4; ++j) {
           float f[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[8 * j + i]) * scale;
+          for (int i = 0; i < 8; ++i) f[i] = fmaf(__uint_as_float(v[8 * j + i]), scale, -shift);
           store_vec<__nv_bfloat16>(
               reinterpret_cast<__nv_bfloat16*>(sb + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)),
               f);
@@ -472,32 +473,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
+        // Pass 1: the row's maximum over this tile (base-2 units) and the
+        // cached entries' cross term, from the fp32 accumulator.
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (c == kBN / 32 - 1) release(buf);
           const int cb = col0 + c * 32;
           const int nvalid = p.cols_valid - cb;  // columns < V in this slab
-          float cm = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(v[i]) * s2;
-            cm = fmaxf(cm, i < nvalid ? x : -INFINITY);
-          }
-          if (cm > -INFINITY) {
-            const float nm = fmaxf(mx, cm);
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(v[i]) * s2;
-              acc += i < nvalid ? ex2_approx(x - nm) : 0.f;
-            }
-            se = se * ex2_approx(mx - nm) + acc;
-            mx = nm;
-          }
+          for (int i = 0; i < 32; ++i)
+            mx = fmaxf(mx, i < nvalid ? __uint_as_float(v[i]) * s2 : -INFINITY);
           while (gcol < cb + 32) {  // cached entries inside this 32-column slab
             const int k = gcol - cb;
             float val = 0.f;
@@ -507,8 +495,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ++gi;
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
-          if (p.store && cb < p.cols_valid)
-            store_box(v, rscale, cb, row0, kElemF32, false, warp_rows);
+        }
+        // Pass 2: sum of 2^(x - max), and the stored logits shifted by the tile
+        // maximum (s~ - max): the entries that carry the probability mass sit
+        // near 0, where the stored value's rounding error vanishes.  Readers
+        // add the maximum back from the tile statistics.
+        const float shift = (p.partials != nullptr && mx > -INFINITY) ? mx * 0.6931471805599453f
+                                                                       : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (c == kBN / 32 - 1) release(buf);
+          const int cb = col0 + c * 32;
+          const int nvalid = p.cols_valid - cb;
+          if (nvalid <= 0) continue;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            se += i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
+          if (p.store) store_box(v, rscale, shift, cb, row0, kElemF32, false, warp_rows);
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
@@ -563,7 +570,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(round_tf32_dev(__uint_as_float(v[i])));
           }
-          store_box(v, 1.f, cb, row0, kElemF32, false, warp_rows);
+          store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows);
         }
       } else {
 #pragma unroll 1
@@ -576,9 +583,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int cb = col0 + c * 32;
           if (cb >= p.cols_valid) continue;
           if (EPI == EPI_STORE)
-            store_box(v, 1.f, cb, row0, kElemF32, false, warp_rows);
+            store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows);
           else  // EPI_ACCUM, fp32 out; K-part ks writes its own block of output rows
-            store_box(v, 1.f, cb, row0 + ur.ks * p.split_rows, true, p.beta != 0, warp_rows);
+            store_box(v, 1.f, 0.f, cb, row0 + ur.ks * p.split_rows, true, p.beta != 0, warp_rows);
         }
       }
     }

@@ -269,6 +269,13 @@ __device__ __forceinline__ float grad_coef(const uint8_t* mask, int row, const S
   return (keep && norm > 0.f) ? g / norm * invT : 0.f;
 }
 
+// The logits epilogue stores s~ minus the row's maximum over the 256-column
+// tile when it also records that tile's statistics (part != nullptr); this is
+// the maximum to add back (base-2 units in part.x), or 0.
+__device__ __forceinline__ float tile_max2(const float4* part, int row, int tiles_n, int col) {
+  return part != nullptr ? part[static_cast<int64_t>(row) * tiles_n + (col >> 8)].x : 0.f;
+}
+
 // dS for the top-K loss, in place over the chunk's logit buffer (one CTA per
 // row):  dS_j = c (m p_s,j - q_j [j in S]),  c = g / (n T),  p_s = exp(s~ - lse).
 // The K cached positions are read before the dense pass and rewritten after it.
@@ -278,7 +285,8 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
                                     const float2* __restrict__ rowinfo,
                                     const int* __restrict__ sidx, const float* __restrict__ sq,
                                     int K, const Scalars* sc, const float* g_dev, float g_host,
-                                    float invT, const float* __restrict__ T_row) {
+                                    float invT, const float* __restrict__ T_row,
+                                    const float4* __restrict__ part, int tiles_n) {
   extern __shared__ float sval[];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
@@ -291,20 +299,24 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   }
   const int* ri = sidx + static_cast<int64_t>(row) * K;
   const float* rq = sq + static_cast<int64_t>(row) * K;
+  const float l2 = lse[row] * kLog2e;
+  // sval[i]: base-2 exponent of p_s at cached entry i, read before the dense pass
   for (int i = threadIdx.x; i < K; i += blockDim.x) {
     const int j = ri[i];
-    sval[i] = j != kEmpty ? to_f<Elem>(srow[j]) : 0.f;
+    sval[i] = j != kEmpty
+                  ? fmaf(to_f<Elem>(srow[j]), kLog2e, tile_max2(part, row, tiles_n, j) - l2)
+                  : 0.f;
   }
   __syncthreads();
   const float m = rowinfo[row].x;
-  const float l2 = lse[row] * kLog2e;
   const float cm = coef * m;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float f[8];
     load8<Elem>(srow + v * 8, f);
+    const float off = tile_max2(part, row, tiles_n, v * 8) - l2;  // 8 | 256: one tile
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      f[i] = (v * 8 + i < V) ? operand_round<Elem>(cm * ex2_approx(fmaf(f[i], kLog2e, -l2)))
+      f[i] = (v * 8 + i < V) ? operand_round<Elem>(cm * ex2_approx(fmaf(f[i], kLog2e, off)))
                              : 0.f;
     store8<Elem>(srow + v * 8, f);
   }
@@ -312,8 +324,7 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   for (int i = threadIdx.x; i < K; i += blockDim.x) {
     const int j = ri[i];
     if (j != kEmpty)
-      srow[j] = from_f<Elem>(
-          operand_round<Elem>(coef * (m * ex2_approx(fmaf(sval[i], kLog2e, -l2)) - rq[i])));
+      srow[j] = from_f<Elem>(operand_round<Elem>(coef * (m * ex2_approx(sval[i]) - rq[i])));
   }
 }
 
@@ -348,7 +359,9 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
                                     const uint8_t* __restrict__ mask, const Scalars* sc,
                                     const float* g_dev, float g_host, float invT,
                                     const float* __restrict__ T_row,
-                                    float* __restrict__ row_loss, int write_grad, float beta) {
+                                    float* __restrict__ row_loss, int write_grad, float beta,
+                                    const float4* __restrict__ part_s,
+                                    const float4* __restrict__ part_t, int tiles_n) {
   __shared__ float2 red[32];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
@@ -362,13 +375,18 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
     float fs[8], ft[8];
     load8<Elem>(srow + v * 8, fs);
     load8<Elem>(trow + v * 8, ft);
+    // stored values are shifted by their tile maxima (8 | 256: one tile per vector)
+    const float ms2 = tile_max2(part_s, row, tiles_n, v * 8);
+    const float mt2 = tile_max2(part_t, row, tiles_n, v * 8);
+    const float dshift = (mt2 - ms2) * kLn2;  // (t~ - s~) = (ft - fs) + dshift
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const bool in = v * 8 + i < V;
-      const float pt = ex2_approx(fmaf(ft[i], kLog2e, -lt2));
-      const float ps = ex2_approx(fmaf(fs[i], kLog2e, -ls2));
-      A += in ? pt * (ft[i] - fs[i]) : 0.f;
-      U += in ? ps * (fs[i] - ft[i]) : 0.f;
+      const float pt = ex2_approx(fmaf(ft[i], kLog2e, mt2 - lt2));
+      const float ps = ex2_approx(fmaf(fs[i], kLog2e, ms2 - ls2));
+      const float u = (fs[i] - ft[i]) - dshift;  // s~ - t~
+      A -= in ? pt * u : 0.f;
+      U += in ? ps * u : 0.f;
       fs[i] = in ? operand_round<Elem>(coef * (ps - pt)) : 0.f;
     }
     if (write_grad && single) store8<Elem>(srow + v * 8, fs);
@@ -381,12 +399,15 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
       float fs[8], ft[8];
       load8<Elem>(srow + v * 8, fs);
       load8<Elem>(trow + v * 8, ft);
+      const float ms2 = tile_max2(part_s, row, tiles_n, v * 8);
+      const float mt2 = tile_max2(part_t, row, tiles_n, v * 8);
+      const float dshift = (mt2 - ms2) * kLn2;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const bool in = v * 8 + i < V;
-        const float pt = ex2_approx(fmaf(ft[i], kLog2e, -lt2));
-        const float ps = ex2_approx(fmaf(fs[i], kLog2e, -ls2));
-        const float g = cf * (ps - pt) + cr * ps * ((fs[i] - ft[i]) - ubar);
+        const float pt = ex2_approx(fmaf(ft[i], kLog2e, mt2 - lt2));
+        const float ps = ex2_approx(fmaf(fs[i], kLog2e, ms2 - ls2));
+        const float g = cf * (ps - pt) + cr * ps * (((fs[i] - ft[i]) - dshift) - ubar);
         fs[i] = in ? operand_round<Elem>(g) : 0.f;
       }
       store8<Elem>(srow + v * 8, fs);

@@ -315,3 +315,39 @@ def test_non_positive_per_token_temperature_sets_status():
     Tr[17] = 0.0
     out = ops.kl_fwd_bwd(w.H, w.W, **dict(_kw(w), T=Tr))
     assert ops.status(out["workspace"]) == 10  # KL_ERR_ARG
+
+
+def test_max_cache_size_K1024():
+    w = wl.make_topk("k1024", N=130, d=64, V=2000, K=1024, d_t=32, T=1.2,
+                     dtype=torch.bfloat16, w_std=0.1, tw_std=0.2, seed=32).to("cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, **_kw(w, chunk=64))
+    assert ops.status(out["workspace"]) == 0
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+@pytest.mark.parametrize("mode", ["topk", "hidden"])
+def test_vocabulary_smaller_than_one_tile(mode):
+    if mode == "topk":
+        w = wl.make_topk("v40", N=70, d=32, V=40, K=40, d_t=16, T=0.9, dtype=torch.bfloat16,
+                         w_std=0.2, tw_std=0.3, seed=33).to("cuda")
+    else:
+        w = wl.make_hidden("v40h", N=70, d=32, d_t=16, V=40, T=0.9, dtype=torch.bfloat16,
+                           w_std=0.2, tw_std=0.3, seed=33).to("cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w))
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+def test_split_backward_accumulates_into_dW():
+    w = _small_topk(seed=34)
+    kw = _kw(w, chunk=128)
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    base = torch.randn(w.W.shape, device="cuda", dtype=torch.float32)
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], dW=base.clone(), accumulate_dW=True, **kw)
+    ref = _oracle(w)
+    _check_grad(b["dW"] - base, ref["dW"], "accumulated dW (split)")
