@@ -283,42 +283,54 @@ def gpu_arm(args):
     if ws > 1:
         ms = max_over_ranks(ms)
 
-    # ---- end to end through the public API: pinned host inputs in, loss out
+    # ---- end to end through the public API: pinned host inputs in, loss out.
+    # Per-step inputs (hidden states, the teacher side, the mask) come from
+    # pinned host memory every step; the heads stay resident (parameters).  A
+    # double-buffered stager copies step i+1's inputs on its own stream while
+    # step i's kernels run, and every step's loss is read back to pinned host
+    # memory.  All copies of the K steps lie inside the timed region.
     e2e = None
     if not args.no_e2e:
-        # per-step inputs: hidden states and the teacher side (cache or teacher
-        # hidden states) and the mask; the heads stay resident (parameters)
+        from chunked_kl_loss_tma_b200.staging import HostStager
+
         names = ["H", "mask", "topk_idx", "topk_logit", "teacher_lse", "Ht"]
         host = {k: getattr(w, k).cpu().pin_memory() for k in names if getattr(w, k) is not None}
-        devb = {k: torch.empty_like(getattr(w, k)) for k in host}
-        hloss = torch.empty((), dtype=torch.float32).pin_memory()
-        kw2 = problem_kwargs(w, args.chunk, override=devb)
-        if args.reverse_weight > 0:
-            kw2["reverse_weight"] = args.reverse_weight
-        prob2, keep2 = ops.make_problem(devb["H"], w.W, **kw2)
+        stager = HostStager(host, dev, depth=2)
+        probs = []
+        for slot in range(stager.depth):
+            kw2 = problem_kwargs(w, args.chunk, override=stager.bufs[slot])
+            if args.reverse_weight > 0:
+                kw2["reverse_weight"] = args.reverse_weight
+            probs.append(ops.make_problem(stager.bufs[slot]["H"], w.W, **kw2))
+        hloss = torch.empty(max(args.steps, 3), dtype=torch.float32).pin_memory()
+        cstream = torch.cuda.current_stream(dev)
 
-        def e2e_step():
-            for k in host:
-                devb[k].copy_(host[k], non_blocking=True)
-            _lib.check(_lib.kl_fwd_bwd(prob2, workspace.data_ptr(), ws_bytes, 1.0,
-                                       loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(), 0,
-                                       stream), "kl_fwd_bwd")
-            hloss.copy_(loss, non_blocking=True)
+        def e2e_run(n):
+            slot = stager.put(host)
+            for i in range(n):
+                stager.acquire(slot, cstream)
+                nxt = stager.put(host) if i + 1 < n else None
+                _lib.check(_lib.kl_fwd_bwd(probs[slot][0], workspace.data_ptr(), ws_bytes, 1.0,
+                                           loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(),
+                                           0, stream), "kl_fwd_bwd")
+                stager.release(slot, cstream)
+                hloss[i].copy_(loss, non_blocking=True)
+                slot = nxt
 
-        for _ in range(3):
-            e2e_step()
+        e2e_run(3)
         barrier()
         e0.record()
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_run(args.steps)
         e1.record()
         barrier()
         ems = e0.elapsed_time(e1)
         if ws > 1:
             ems = max_over_ranks(ems)
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
         e2e = {"value": ws * args.N * args.steps / (ems / 1e3),
-               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+               "unit": "tokens/s", "h2d_bytes_per_step": stager.bytes_per_step,
+               "d2h_bytes_per_step": 4,
+               "pipeline": "inputs double-buffered: step i+1's host-to-device copy overlaps "
+                           "step i's kernels; loss read back every step"}
 
     if ws > 1:
         dist.barrier()

@@ -39,8 +39,8 @@ def _need(t, name, dtype=None, device=None):
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
                  Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0):
-    """T: a number, or a float32 tensor [N] of per-token temperatures."""
-    """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive)."""
+    """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive).
+    T: a number, or a float32 tensor [N] of per-token temperatures."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
     dev = H.device
