@@ -28,7 +28,8 @@ KL_NOALLOC_SCRATCH_BYTES = 16 << 20
 # Every symbol declared in include/chunked_kl.h.
 EXPORTS = ("kl_workspace_bytes", "kl_fwd", "kl_bwd", "kl_fwd_bwd", "kl_status",
            "kl_status_string", "kl_launch_count", "kl_profile_begin", "kl_profile_end",
-           "kl_fwd_noalloc")
+           "kl_fwd_noalloc", "kl_vp_num_chunks", "kl_vp_fwd_chunk", "kl_vp_bwd_chunk",
+           "kl_cast_f32")
 
 
 class KLProblem(ctypes.Structure):
@@ -42,6 +43,7 @@ class KLProblem(ctypes.Structure):
         ("d_t", ctypes.c_int64), ("Ht", ctypes.c_void_p), ("Wt", ctypes.c_void_p),
         ("chunk_tokens", ctypes.c_int64), ("normalizer", ctypes.c_float),
         ("reverse_weight", ctypes.c_float), ("T_row", ctypes.c_void_p),
+        ("v_begin", ctypes.c_int64), ("V_total", ctypes.c_int64),
     ]
 
 
@@ -81,6 +83,15 @@ def lib():
     L.kl_fwd_bwd.restype = i32
     L.kl_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
     L.kl_fwd_noalloc.restype = i32
+    i64 = ctypes.c_int64
+    L.kl_vp_num_chunks.argtypes = [P]
+    L.kl_vp_num_chunks.restype = i64
+    L.kl_vp_fwd_chunk.argtypes = [P, i64, vp, sz, vp, vp]
+    L.kl_vp_fwd_chunk.restype = i32
+    L.kl_vp_bwd_chunk.argtypes = [P, i64, vp, sz, vp, i32, i32, f32, vp, vp, vp, vp, vp, i32, vp]
+    L.kl_vp_bwd_chunk.restype = i32
+    L.kl_cast_f32.argtypes = [vp, vp, i64, i32, vp]
+    L.kl_cast_f32.restype = i32
     L.kl_status.argtypes = [vp, vp]
     L.kl_status.restype = i32
     L.kl_status_string.argtypes = [i32]
@@ -129,6 +140,25 @@ def kl_fwd_noalloc(prob, loss, lse_s, row_loss, status, stream):
     """Forward with the library's fixed static scratch instead of a workspace,
     for callers that cannot allocate device memory (see include/chunked_kl.h)."""
     return lib().kl_fwd_noalloc(ctypes.byref(prob), loss, lse_s, row_loss, status, stream)
+
+
+def kl_vp_num_chunks(prob):
+    return int(lib().kl_vp_num_chunks(ctypes.byref(prob)))
+
+
+def kl_vp_fwd_chunk(prob, chunk, ws, ws_bytes, row_stats, stream):
+    return lib().kl_vp_fwd_chunk(ctypes.byref(prob), int(chunk), ws, ws_bytes, row_stats, stream)
+
+
+def kl_vp_bwd_chunk(prob, chunk, ws, ws_bytes, row_stats_all, P, rank, grad_loss, loss, lse_s,
+                    row_loss, dH_part, dW, accumulate_dW, stream):
+    return lib().kl_vp_bwd_chunk(ctypes.byref(prob), int(chunk), ws, ws_bytes, row_stats_all,
+                                 int(P), int(rank), float(grad_loss), loss, lse_s, row_loss,
+                                 dH_part, dW, int(accumulate_dW), stream)
+
+
+def kl_cast_f32(src, dst, n, dtype, stream):
+    return lib().kl_cast_f32(src, dst, int(n), int(dtype), stream)
 
 
 def kl_status(ws, stream):

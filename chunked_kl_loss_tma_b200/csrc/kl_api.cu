@@ -242,6 +242,9 @@ int validate_shape(const kl_problem* p) {
   if (!(p->reverse_weight >= 0.f && p->reverse_weight <= 1.f) ||
       (p->reverse_weight > 0.f && p->teacher != KL_TEACHER_HIDDEN))
     return KL_ERR_ARG;
+  if (p->v_begin < 0 || p->V_total < 0 || p->V_total > (int64_t(1) << 31) - 512 ||
+      (p->V_total > 0 && p->v_begin + p->V > p->V_total) || (p->V_total == 0 && p->v_begin != 0))
+    return KL_ERR_ARG;
   if (p->d % 8 != 0) return KL_ERR_ALIGN;
   if (p->teacher == KL_TEACHER_TOPK) {
     if (p->K < 1 || p->K > kMaxK) return KL_ERR_SHAPE;
@@ -268,6 +271,11 @@ int validate(const kl_problem* p) {
   }
   return KL_OK;
 }
+
+// Rows of the whole head (the vocabulary the cache ids index).
+int64_t vocab_total(const kl_problem* p) { return p->V_total > 0 ? p->V_total : p->V; }
+// The problem covers the whole head (every call except kl_vp_*).
+bool whole_head(const kl_problem* p) { return p->v_begin == 0 && vocab_total(p) == p->V; }
 
 Plan make_plan(const kl_problem* p, int entry) {
   Plan pl;
@@ -549,8 +557,10 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
                                                  2.0 * Cn * p->V * dx);
 }
 
+// dH_f32: write dH as fp32 (a vocabulary shard's partial sum) whatever Elem is.
 template <typename Elem>
-int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta) {
+int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+               bool dH_f32 = false) {
   if (sizeof(Elem) == 4)
     return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
   const kl_problem* p = c.p;
@@ -591,10 +601,23 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
         return KL_ERR_CUDA;
       KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
-      LaunchScope ls("splitk_reduce", c.st, 0, (4.0 * ks + sizeof(Elem)) * Cn * d);
-      splitk_reduce_kernel<Elem><<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(
-          part, ks, rows_pad * d, static_cast<Elem*>(dH) + c0 * d, Cn * d);
+      LaunchScope ls("splitk_reduce", c.st, 0,
+                     (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
+      if (dH_f32)
+        splitk_reduce_kernel<float><<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(
+            part, ks, rows_pad * d, static_cast<float*>(dH) + c0 * d, Cn * d);
+      else
+        splitk_reduce_kernel<Elem><<<static_cast<unsigned>(c.sms * 8), 256, 0, c.st>>>(
+            part, ks, rows_pad * d, static_cast<Elem*>(dH) + c0 * d, Cn * d);
       KL_TRY(cudaGetLastError() == cudaSuccess ? KL_OK : KL_ERR_CUDA);
+    } else if (dH_f32) {
+      // fp32 store straight into the chunk's rows (boxes past row Cn are clipped)
+      gp.beta = 0;
+      CUtensorMap mc;
+      if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
+        return KL_ERR_CUDA;
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
+                                                    2.0 * Cn * p->V * d)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
@@ -655,8 +678,8 @@ int launch_prep(Ctx& c, int64_t c0, int64_t Cn) {
                      c.st>>>(p->topk_idx + c0 * K, p->topk_logit + c0 * K,
                              p->teacher_lse ? p->teacher_lse + c0 : nullptr, c.invT,
                              p->T_row ? p->T_row + c0 : nullptr,
-                             static_cast<int>(p->V), K, static_cast<int>(Cn), sidx, sq, rinfo,
-                             c.sc);
+                             static_cast<int>(vocab_total(p)), K, static_cast<int>(Cn), sidx, sq,
+                             rinfo, c.sc, static_cast<int>(p->v_begin), static_cast<int>(p->V));
   return KL_LAUNCHED();
 }
 
@@ -668,7 +691,18 @@ int launch_row_reduce(Ctx& c, const float4* partials, int64_t c0, int64_t Cn, bo
   LaunchScope ls("row_reduce", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 16);
   row_reduce_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
       partials, c.pl.tiles_v, static_cast<int>(Cn), p->mask ? p->mask + c0 : nullptr, rinfo,
-      lse_out + c0, row_loss ? row_loss + c0 : nullptr);
+      lse_out + c0, row_loss ? row_loss + c0 : nullptr, 1, nullptr);
+  return KL_LAUNCHED();
+}
+
+// A vocabulary shard's row statistics, interleaved pairs: lse -> out[2 i + slot],
+// and in top-K mode the cross term -> out[2 i + 1].
+int launch_row_stats(Ctx& c, const float4* partials, int64_t Cn, float* out, int slot,
+                     bool cross) {
+  LaunchScope ls("row_reduce", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 16);
+  row_reduce_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
+      partials, c.pl.tiles_v, static_cast<int>(Cn), nullptr, nullptr, out + slot, nullptr, 2,
+      cross ? out + 1 : nullptr);
   return KL_LAUNCHED();
 }
 
@@ -698,7 +732,7 @@ template <typename Elem>
 int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
                         const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
                         float* row_loss, int write_grad, const float4* part_s,
-                        const float4* part_t) {
+                        const float4* part_t, int add_lse = 1) {
   const kl_problem* p = c.p;
   LaunchScope ls("dlogits_full", c.st, 0,
                  ((write_grad ? 3.0 : 2.0) + (p->reverse_weight > 0.f && write_grad ? 2.0 : 0.0)) *
@@ -707,7 +741,7 @@ int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
       S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
       p->T_row ? p->T_row + c0 : nullptr, row_loss ? row_loss + c0 : nullptr, write_grad,
-      p->reverse_weight, part_s, part_t, c.pl.tiles_v);
+      p->reverse_weight, part_s, part_t, c.pl.tiles_v, add_lse);
   return KL_LAUNCHED();
 }
 
@@ -724,8 +758,10 @@ int launch_fill(Ctx& c, float* p, int64_t n, float v) {
   return KL_LAUNCHED();
 }
 
-int begin(const kl_problem* p, int entry, void* ws, size_t ws_bytes, void* stream, Ctx& c) {
+int begin(const kl_problem* p, int entry, void* ws, size_t ws_bytes, void* stream, Ctx& c,
+          bool vocab_shard = false) {
   KL_TRY(validate(p));
+  if (!vocab_shard && !whole_head(p)) return KL_ERR_ARG;
   DevInfo di;
   KL_TRY(current_device_info(&di));
   c.p = p;
@@ -850,6 +886,91 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
   return launch_finalize(c, rl, loss);
 }
 
+// ------------------------------------------------------------------ vocabulary-parallel chunks
+// Rows [c0, c0 + Cn) of chunk k.
+void chunk_rows(const Ctx& c, int64_t k, int64_t* c0, int64_t* Cn) {
+  *c0 = k * c.pl.C;
+  const int64_t left = c.p->N - *c0;
+  *Cn = left < c.pl.C ? left : c.pl.C;
+}
+
+int64_t num_chunks(const kl_problem* p, int64_t C) { return p->N > 0 ? cdiv(p->N, C) : 0; }
+
+template <typename Elem>
+int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
+  const kl_problem* p = c.p;
+  int64_t c0, Cn;
+  chunk_rows(c, k, &c0, &Cn);
+  if (k == 0) {  // start of a pass
+    KL_TRY(launch_count_valid(c));
+    KL_TRY(prepare_heads(c));
+    if (sizeof(Elem) == 4)
+      KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
+                              reinterpret_cast<float*>(c.ws + c.pl.off_wT), c.pl.Vp, p->V, p->d));
+  }
+  Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  if (!c.pl.hidden) {
+    KL_TRY(launch_prep(c, c0, Cn));
+    KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps,
+                             reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+                             reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
+                             "gemm_logits_stats"));
+    return launch_row_stats(c, ps, Cn, stats, 0, true);
+  }
+  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
+  float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+  KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
+                           "gemm_logits_stats"));
+  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
+                           "gemm_teacher_logits"));
+  KL_TRY(launch_row_stats(c, ps, Cn, stats, 0, false));
+  return launch_row_stats(c, pt, Cn, stats, 1, false);
+}
+
+template <typename Elem>
+int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank, float g,
+                     float* loss, float* lse_user, float* row_loss, float* dH, float* dW,
+                     int accumulate) {
+  const kl_problem* p = c.p;
+  int64_t c0, Cn;
+  chunk_rows(c, k, &c0, &Cn);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(c.ws + c.pl.off_rl);
+  float* lse_s = reinterpret_cast<float*>(c.ws + c.pl.off_lse_s);
+  float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
+  Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  {
+    LaunchScope ls("vp_merge", c.st, 0, static_cast<double>(Cn) * (8.0 * P + 12));
+    vp_merge_kernel<<<static_cast<unsigned>(cdiv(Cn, 128)), 128, 0, c.st>>>(
+        stats_all, P, static_cast<int>(Cn), c.pl.hidden ? 1 : 0, rank,
+        p->mask ? p->mask + c0 : nullptr,
+        c.pl.hidden ? nullptr : reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
+        lse_s + c0, lse_t ? lse_t + c0 : nullptr, lse_user ? lse_user + c0 : nullptr, rl + c0);
+    KL_TRY(KL_LAUNCHED());
+  }
+  if (!c.pl.hidden) {
+    KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
+  } else {
+    Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
+    float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+    KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1, ps, pt,
+                                     rank == 0 ? 1 : 0));
+  }
+  KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || k > 0) ? 1 : 0, true));
+  if (c0 + Cn == p->N) KL_TRY(launch_finalize(c, rl, loss));
+  return KL_OK;
+}
+
+// Checks shared by the two vocabulary-parallel calls.
+int vp_begin(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes, void* stream,
+             Ctx& c) {
+  KL_TRY(validate(p));
+  if (p->reverse_weight != 0.f) return KL_ERR_ARG;
+  if (chunk < 0 || chunk >= num_chunks(p, make_plan(p, KL_ENTRY_FWD_BWD).C)) return KL_ERR_ARG;
+  return begin(p, KL_ENTRY_FWD_BWD, ws, ws_bytes, stream, c, true);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -897,6 +1018,57 @@ int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss, 
   return p->dtype == KL_DTYPE_BF16
              ? run_fwd_bwd<__nv_bfloat16>(c, grad_loss, loss, row_loss, dH, dW, accumulate_dW)
              : run_fwd_bwd<float>(c, grad_loss, loss, row_loss, dH, dW, accumulate_dW);
+}
+
+int64_t kl_vp_num_chunks(const kl_problem* p) {
+  if (validate_shape(p) != KL_OK) return -1;
+  return num_chunks(p, make_plan(p, KL_ENTRY_FWD_BWD).C);
+}
+
+int kl_vp_fwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    float* row_stats, void* stream) {
+  Ctx c;
+  KL_TRY(vp_begin(p, chunk, ws, ws_bytes, stream, c));
+  if (row_stats == nullptr) return KL_ERR_NULL;
+  return p->dtype == KL_DTYPE_BF16 ? run_vp_fwd_chunk<__nv_bfloat16>(c, chunk, row_stats)
+                                   : run_vp_fwd_chunk<float>(c, chunk, row_stats);
+}
+
+int kl_vp_bwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    const float* row_stats_all, int P, int rank, float grad_loss, float* loss,
+                    float* lse_s, float* row_loss, float* dH_part, float* dW, int accumulate_dW,
+                    void* stream) {
+  if (P < 1 || rank < 0 || rank >= P) return KL_ERR_ARG;
+  Ctx c;
+  KL_TRY(vp_begin(p, chunk, ws, ws_bytes, stream, c));
+  if (row_stats_all == nullptr || loss == nullptr || dH_part == nullptr || dW == nullptr)
+    return KL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(dH_part) | reinterpret_cast<uintptr_t>(dW)) & 15)
+    return KL_ERR_ALIGN;
+  return p->dtype == KL_DTYPE_BF16
+             ? run_vp_bwd_chunk<__nv_bfloat16>(c, chunk, row_stats_all, P, rank, grad_loss, loss,
+                                               lse_s, row_loss, dH_part, dW, accumulate_dW)
+             : run_vp_bwd_chunk<float>(c, chunk, row_stats_all, P, rank, grad_loss, loss, lse_s,
+                                       row_loss, dH_part, dW, accumulate_dW);
+}
+
+int kl_cast_f32(const float* src, void* dst, int64_t n, int dtype, void* stream) {
+  if (n < 0 || n % 4 != 0) return KL_ERR_SHAPE;
+  if (dtype != KL_DTYPE_BF16 && dtype != KL_DTYPE_F32) return KL_ERR_DTYPE;
+  if (n == 0) return KL_OK;
+  if (src == nullptr || dst == nullptr) return KL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15)
+    return KL_ERR_ALIGN;
+  DevInfo di;
+  KL_TRY(current_device_info(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LaunchScope ls("cast_f32", st, 0, n * (dtype == KL_DTYPE_BF16 ? 6.0 : 8.0));
+  const unsigned grid = static_cast<unsigned>(di.sms * 4);
+  if (dtype == KL_DTYPE_BF16)
+    cast_f32_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), n);
+  else
+    cast_f32_kernel<float><<<grid, 256, 0, st>>>(src, static_cast<float*>(dst), n);
+  return KL_LAUNCHED();
 }
 
 int kl_status(void* ws, void* stream) {
@@ -1000,6 +1172,7 @@ int noalloc_scratch(uint8_t** out) {
 extern "C" int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
                               int* status, void* stream) {
   KL_TRY(validate(p));
+  if (!whole_head(p)) return KL_ERR_ARG;
   if (p->dtype != KL_DTYPE_BF16 || p->teacher != KL_TEACHER_TOPK) return KL_ERR_DTYPE;
   if (loss == nullptr || (p->N > 0 && (lse_s == nullptr || row_loss == nullptr)))
     return KL_ERR_NULL;

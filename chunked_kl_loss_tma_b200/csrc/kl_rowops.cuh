@@ -152,13 +152,19 @@ __global__ void count_valid_kernel(const uint8_t* mask, int64_t N, float normali
 // probabilities on the support:
 //   partial mass (lse_t != nullptr): q = exp(t / T - lse_t)
 //   renormalised:                    q = softmax over valid entries of t / T
-// rowinfo = (m = sum q, sum q log q).
+// rowinfo = (m = sum q, sum q log q), over all cached entries.
+// Ids are vocabulary ids in [0, V_total).  The sorted ids are stored relative
+// to this head's first row v_begin; entries outside [v_begin, v_begin + V_local)
+// (another rank's vocabulary shard) become kBelow / kEmpty, so the sorted order
+// holds and no column of this shard ever matches them.
+constexpr int kBelow = static_cast<int>(0x80000000u);
 __global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
                                  const float* __restrict__ logit,
                                  const float* __restrict__ lse_t, float invT,
                                  const float* __restrict__ T_row, int V, int K, int rows,
                                  int* __restrict__ sidx, float* __restrict__ sq,
-                                 float2* __restrict__ rowinfo, Scalars* sc) {
+                                 float2* __restrict__ rowinfo, Scalars* sc, int v_begin,
+                                 int V_local) {
   extern __shared__ int prep_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -219,7 +225,10 @@ __global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
       rank += (kj < ki) || (kj == ki && j < i);
       bad |= (kj == ki && j != i && ki != kEmpty);
     }
-    so[rank] = ki;
+    so[rank] = ki == kEmpty ? kEmpty
+               : ki < v_begin ? kBelow
+               : ki - v_begin >= V_local ? kEmpty
+                                         : ki - v_begin;
     qo[rank] = qv[i];
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(&sc->status, 0, kStatusIndex);
@@ -227,12 +236,15 @@ __global__ void prep_topk_kernel(const int32_t* __restrict__ idx,
 }
 
 // Split-V merge (one warp per row): partials (max2, sumexp2, cross) of every
-// 256-column tile -> lse = ln 2 * (M + log2 Z).  In top-K mode also the row
-// loss l = [sum q log q] - [sum q s~] + m * lse (0 on masked rows).
+// 256-column tile -> lse = ln 2 * (M + log2 Z), written to lse_out[row * stride].
+// In top-K mode also the row loss l = [sum q log q] - [sum q s~] + m * lse
+// (0 on masked rows) when row_loss is given, and the cross term sum q s~ to
+// cross_out[row * stride] when that is given (a vocabulary shard's statistics).
 __global__ void row_reduce_kernel(const float4* __restrict__ partials, int tiles_n, int rows,
                                   const uint8_t* __restrict__ mask,
                                   const float2* __restrict__ rowinfo, float* __restrict__ lse_out,
-                                  float* __restrict__ row_loss) {
+                                  float* __restrict__ row_loss, int stride,
+                                  float* __restrict__ cross_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= rows) return;
@@ -250,7 +262,8 @@ __global__ void row_reduce_kernel(const float4* __restrict__ partials, int tiles
   cross = warp_sum(cross);
   if (lane == 0) {
     const float lse = (M + log2f(Z)) * kLn2;
-    lse_out[row] = lse;
+    lse_out[static_cast<int64_t>(row) * stride] = lse;
+    if (cross_out != nullptr) cross_out[static_cast<int64_t>(row) * stride] = cross;
     if (rowinfo != nullptr && row_loss != nullptr) {
       const bool keep = mask == nullptr || mask[row] != 0;
       const float2 ri = rowinfo[row];
@@ -302,8 +315,8 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   const float l2 = lse[row] * kLog2e;
   // sval[i]: base-2 exponent of p_s at cached entry i, read before the dense pass
   for (int i = threadIdx.x; i < K; i += blockDim.x) {
-    const int j = ri[i];
-    sval[i] = j != kEmpty
+    const int j = ri[i];  // in [0, V): a cached column of this head; else empty or elsewhere
+    sval[i] = static_cast<unsigned>(j) < static_cast<unsigned>(V)
                   ? fmaf(to_f<Elem>(srow[j]), kLog2e, tile_max2(part, row, tiles_n, j) - l2)
                   : 0.f;
   }
@@ -323,7 +336,7 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   __syncthreads();
   for (int i = threadIdx.x; i < K; i += blockDim.x) {
     const int j = ri[i];
-    if (j != kEmpty)
+    if (static_cast<unsigned>(j) < static_cast<unsigned>(V))
       srow[j] = from_f<Elem>(operand_round<Elem>(coef * (m * ex2_approx(sval[i]) - rq[i])));
   }
 }
@@ -361,7 +374,8 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
                                     const float* __restrict__ T_row,
                                     float* __restrict__ row_loss, int write_grad, float beta,
                                     const float4* __restrict__ part_s,
-                                    const float4* __restrict__ part_t, int tiles_n) {
+                                    const float4* __restrict__ part_t, int tiles_n,
+                                    int add_lse) {
   __shared__ float2 red[32];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
@@ -415,9 +429,67 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
   }
   if (threadIdx.x == 0 && row_loss != nullptr) {
     const bool keep = mask == nullptr || mask[row] != 0;
-    const float fwd = r.x - lse_t[row] + lse_s[row];
-    const float rev = ubar - lse_s[row] + lse_t[row];
+    // add_lse = 0: a vocabulary shard's share, the sums over its columns only
+    const float dl = add_lse ? lse_s[row] - lse_t[row] : 0.f;
+    const float fwd = r.x + dl;
+    const float rev = ubar - dl;
     row_loss[row] = keep ? (1.f - beta) * fwd + beta * rev : 0.f;
+  }
+}
+
+// Vocabulary-parallel merge (one thread per row).  stats holds, for each of P
+// head shards (rank-major blocks of rows x 2 floats), the shard's row
+// statistics: top-K mode (lse over the shard, cross term over the shard's
+// cached entries); teacher-hidden mode (student lse, teacher lse over the
+// shard).  A log-sum-exp over the union of shards is the log of the sum of the
+// shards' exponentials; the cross term is a plain sum.  Shards merge in rank
+// order, so every rank gets the same bits.  Writes the full-vocabulary lse_s
+// (and lse_t) of each row, and in top-K mode the row loss
+// [sum q log q] - cross + m * lse_s on rank 0 and 0 on the others (0 on masked
+// rows), so that the ranks' row losses sum to the loss.
+__global__ void vp_merge_kernel(const float* __restrict__ stats, int P, int rows, int hidden,
+                                int rank, const uint8_t* __restrict__ mask,
+                                const float2* __restrict__ rowinfo, float* __restrict__ lse_s,
+                                float* __restrict__ lse_t, float* __restrict__ lse_copy,
+                                float* __restrict__ row_loss) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  const int64_t blk = static_cast<int64_t>(rows) * 2;
+  float mx = -INFINITY, my = -INFINITY;
+  for (int r = 0; r < P; ++r) {
+    const float* st = stats + r * blk + static_cast<int64_t>(row) * 2;
+    mx = fmaxf(mx, st[0]);
+    my = fmaxf(my, st[1]);
+  }
+  float zx = 0.f, zy = 0.f, cross = 0.f;
+  for (int r = 0; r < P; ++r) {
+    const float* st = stats + r * blk + static_cast<int64_t>(row) * 2;
+    zx += expf(st[0] - mx);
+    if (hidden) zy += expf(st[1] - my);
+    else cross += st[1];
+  }
+  const float ls = mx + logf(zx);
+  lse_s[row] = ls;
+  if (lse_copy != nullptr) lse_copy[row] = ls;
+  if (hidden) {
+    lse_t[row] = my + logf(zy);
+  } else if (row_loss != nullptr) {
+    const bool keep = mask == nullptr || mask[row] != 0;
+    const float2 ri = rowinfo[row];
+    row_loss[row] = (keep && rank == 0) ? (ri.y - cross + ri.x * ls) : 0.f;
+  }
+}
+
+// dst = src converted to Elem, n values (n a multiple of 4).
+template <typename Elem>
+__global__ void cast_f32_kernel(const float* __restrict__ src, Elem* __restrict__ dst, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < (n >> 2);
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(src)[i];
+    dst[4 * i] = from_f<Elem>(a.x);
+    dst[4 * i + 1] = from_f<Elem>(a.y);
+    dst[4 * i + 2] = from_f<Elem>(a.z);
+    dst[4 * i + 3] = from_f<Elem>(a.w);
   }
 }
 

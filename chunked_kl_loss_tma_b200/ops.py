@@ -38,9 +38,12 @@ def _need(t, name, dtype=None, device=None):
 
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
-                 Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0):
+                 Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0,
+                 v_begin=0, V_total=0):
     """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive).
-    T: a number, or a float32 tensor [N] of per-token temperatures."""
+    T: a number, or a float32 tensor [N] of per-token temperatures.
+    v_begin, V_total: W (and Wt) are rows [v_begin, v_begin + V) of a V_total-row
+    head (vocabulary-parallel calls only)."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
     dev = H.device
@@ -69,6 +72,8 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
     p.chunk_tokens = int(chunk_tokens)
     p.normalizer = float(normalizer)
     p.reverse_weight = float(reverse_weight)
+    p.v_begin = int(v_begin)
+    p.V_total = int(V_total)
     keep = [H, W, mask, T_row]
     if Ht is not None:
         _need(Ht, "Ht", H.dtype, dev)

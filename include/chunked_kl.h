@@ -126,6 +126,12 @@ typedef struct kl_problem {
                                 teacher_lse must then be taken at each row's T.
                                 A value <= 0 is flagged as KL_ERR_ARG in the
                                 device status (kl_status).                       */
+  int64_t v_begin;           /* vocabulary-parallel calls (kl_vp_*): W (and Wt)
+                                hold rows [v_begin, v_begin + V) of a head with
+                                V_total rows.  Must be 0 for the other calls.    */
+  int64_t V_total;           /* vocabulary-parallel calls: rows of the whole
+                                head; 0 or V for the other calls.  Cache ids are
+                                always ids of the whole vocabulary.              */
 } kl_problem;
 
 /* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if
@@ -187,6 +193,63 @@ int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss,
 #define KL_NOALLOC_SCRATCH_BYTES (16u << 20)
 int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
                    int* status, void* stream);
+
+/* ---------------------------------------------------------------- vocabulary-parallel form
+ *
+ * The head split by vocabulary rows over P ranks, as in tensor-parallel
+ * training of the output layer (the pages' toy benchmark reports the slowest
+ * tensor-parallel rank, §B "Toy Loss-Kernel Benchmark Configuration").  Rank r
+ * holds W rows [v_begin, v_begin + V) of the V_total-row head (and the same
+ * rows of Wt); H, mask, T / T_row and the teacher side (cache with whole-
+ * vocabulary ids and teacher_lse, or Ht) are identical on every rank.  The
+ * loss is exact: only the log-sum-exp over V needs every shard, and it merges
+ * from per-shard values (log sum_r exp lse_r).  For every token chunk
+ * k = 0 .. kl_vp_num_chunks() - 1, in order, on one workspace (size
+ * kl_workspace_bytes(p, KL_ENTRY_FWD_BWD)):
+ *
+ *   1. kl_vp_fwd_chunk  -> row_stats [rows_k][2] of this shard
+ *   2. the caller gathers all ranks' row_stats, rank-major: [P][rows_k][2]
+ *      (e.g. an NCCL all-gather; 8 bytes per row per rank)
+ *   3. kl_vp_bwd_chunk  -> this rank's share of the row losses and of dH
+ *      (fp32, rows of chunk k), and dW rows of its own shard
+ *
+ * then sums over ranks (e.g. an NCCL all-reduce) the fp32 dH partials, the
+ * loss and, if wanted, row_loss: each rank's value is its share, and the sum
+ * over ranks is the result.  kl_cast_f32 turns the summed fp32 dH into H's
+ * dtype.  rows_k = min(C, N - k C) with C = chunk_tokens (default 4096).
+ * Chunk 0 starts a pass (it resets the status word and prepares the heads);
+ * the workspace carries the chunk's logits from step 1 to step 3, so no other
+ * call may use it in between.  Requires reverse_weight = 0 (the reverse-KL
+ * gradient needs a second per-row exchange; not provided): KL_ERR_ARG.
+ * Errors as kl_fwd_bwd, plus KL_ERR_ARG for v_begin < 0, v_begin + V > V_total,
+ * chunk outside [0, kl_vp_num_chunks()), P < 1 or rank outside [0, P). */
+
+/* Number of token chunks of the pass (0 when N = 0), or -1 if p is invalid. */
+int64_t kl_vp_num_chunks(const kl_problem* p);
+
+/* Step 1 for chunk k: logits of the chunk over this shard (kept in ws) and the
+ * rows' statistics over the shard: row_stats[i] = (lse_s over the shard, cross
+ * term sum_{cached ids in the shard} q s~) in top-K mode, (lse_s, lse_t over the
+ * shard) in teacher-hidden mode.  Tensor work: 2 rows_k d V (+ 2 rows_k d_t V). */
+int kl_vp_fwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    float* row_stats, void* stream);
+
+/* Step 3 for chunk k.  row_stats_all: [P][rows_k][2], every rank's step-1
+ * output in rank order.  Writes lse_s [N] rows of the chunk (whole-vocabulary
+ * student lse; may be NULL), row_loss [N] rows of the chunk (this rank's share;
+ * may be NULL), dH_part [N, d] fp32 rows of the chunk (this rank's share,
+ * dS_shard . W_shard), and dW [V, d] fp32 (this shard's rows; overwritten at
+ * chunk 0 unless accumulate_dW, accumulated otherwise).  After the last chunk
+ * it writes loss (device scalar, this rank's share of the mean).  grad_loss is
+ * the incoming gradient g.  Tensor work: 4 rows_k d V. */
+int kl_vp_bwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    const float* row_stats_all, int P, int rank, float grad_loss, float* loss,
+                    float* lse_s, float* row_loss, float* dH_part, float* dW, int accumulate_dW,
+                    void* stream);
+
+/* dst[i] = src[i] converted to dtype (KL_DTYPE_BF16: round to nearest even;
+ * KL_DTYPE_F32: copy), i < n; n a multiple of 4, both 16-byte aligned. */
+int kl_cast_f32(const float* src, void* dst, int64_t n, int dtype, void* stream);
 
 /* Synchronises stream, then returns the device-side status recorded in ws
  * (KL_OK, KL_ERR_INDEX or KL_ERR_TIMEOUT), or KL_ERR_CUDA if the stream

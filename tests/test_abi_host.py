@@ -22,7 +22,7 @@ def lib():
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_\s\*]*?\b(kl_[a-z_]+)\s*\(",
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_\s\*]*?\b(kl_[a-z0-9_]+)\s*\(",
                        src, flags=re.M)
     return sorted(set(names))
 
@@ -104,3 +104,34 @@ def test_status_strings(lib):
     for code, name in L.STATUS.items():
         assert L.kl_status_string(code) and isinstance(L.kl_status_string(code), str)
     assert lib.kl_launch_count() >= 0
+
+
+def test_vocab_parallel_host_checks(lib):
+    p = _problem(chunk_tokens=1024, v_begin=1024, V=4096, V_total=128256)
+    assert L.kl_vp_num_chunks(p) == 4
+    assert L.kl_vp_num_chunks(_problem(N=0, V_total=128256)) == 0
+    assert L.kl_vp_num_chunks(_problem(v_begin=256, V_total=128256)) == -1   # past the head
+    assert L.kl_vp_num_chunks(_problem(v_begin=-1, V_total=128256)) == -1
+    assert L.kl_vp_num_chunks(_problem(v_begin=8)) == -1                     # shard without V_total
+    p.H = p.W = p.topk_idx = p.topk_logit = 256
+    # the whole-head entry points refuse a shard
+    assert L.kl_fwd_bwd(p, 256, 1 << 40, 1.0, 256, None, 256, 256, 0, None) == 10
+    assert L.kl_fwd(p, 256, 1 << 40, 256, 256, None, None, None) == 10
+    # chunk index, rank and reverse weight are checked before the device
+    assert L.kl_vp_fwd_chunk(p, 4, 256, 1 << 40, 256, None) == 10
+    assert L.kl_vp_fwd_chunk(p, -1, 256, 1 << 40, 256, None) == 10
+    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, 2, 2, 1.0, 256, None, None, 256, 256, 0,
+                             None) == 10
+    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, 0, 0, 1.0, 256, None, None, 256, 256, 0,
+                             None) == 10
+    q = _problem(teacher=1, d_t=4096, K=0, V=4096, V_total=128256, reverse_weight=0.5)
+    q.H = q.W = q.Ht = q.Wt = 256
+    assert L.kl_vp_fwd_chunk(q, 0, 256, 1 << 40, 256, None) == 10
+
+
+def test_cast_host_checks(lib):
+    assert L.kl_cast_f32(256, 256, 6, L.KL_DTYPE_BF16, None) == 2      # n not a multiple of 4
+    assert L.kl_cast_f32(256, 256, 8, 9, None) == 3
+    assert L.kl_cast_f32(None, 256, 8, L.KL_DTYPE_BF16, None) == 1
+    assert L.kl_cast_f32(260, 256, 8, L.KL_DTYPE_BF16, None) == 4
+    assert L.kl_cast_f32(None, None, 0, L.KL_DTYPE_BF16, None) == 0
