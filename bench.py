@@ -51,6 +51,11 @@ def parse():
     ap.add_argument("--entry", default="fused", choices=["fused", "split"],
                     help="fused: kl_fwd_bwd; split: kl_fwd then kl_bwd (the autograd path, "
                          "backward recomputes the logits)")
+    ap.add_argument("--parallel", default="tokens", choices=["tokens", "vocab"],
+                    help="tokens: each rank its own token shard, no collective (weak scaling); "
+                         "vocab: the head split by vocabulary rows over the ranks, the same "
+                         "tokens on every rank, one statistics all-gather per chunk and an "
+                         "all-reduce of dH (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=0,
@@ -210,23 +215,42 @@ def gpu_arm(args):
             dist.init_process_group("nccl", device_id=dev, timeout=_pg_timeout())
         else:
             dist.init_process_group(backend, timeout=_pg_timeout())
-    w = make_workload(wl, args, dev, rank)
+    vocab = args.parallel == "vocab"
+    if vocab and (args.entry != "fused" or args.reverse_weight > 0):
+        raise SystemExit("--parallel vocab runs the fused pass with forward KL only")
+    # vocabulary-parallel ranks share the tokens: the same seed everywhere
+    w = make_workload(wl, args, dev, 0 if vocab else rank)
     args.N = w.N
     torch.cuda.empty_cache()  # drop the teacher-cache generator's temporaries
     kw = problem_kwargs(w, args.chunk)
     if args.reverse_weight > 0:
         kw["reverse_weight"] = args.reverse_weight
-    prob, keep = ops.make_problem(w.H, w.W, **kw)
+    shard = None
+    if vocab:
+        from chunked_kl_loss_tma_b200 import vocab_parallel as vpm
+
+        v0, v1 = vpm.vocab_shard(w.V, ws, rank)
+        W_head = w.W[v0:v1]
+        if w.mode == "hidden":
+            kw["Wt"] = w.Wt[v0:v1]
+        prob, keep = ops.make_problem(w.H, W_head, v_begin=v0, V_total=w.V, **kw)
+    else:
+        W_head = w.W
+        prob, keep = ops.make_problem(w.H, w.W, **kw)
     ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     dH = torch.empty_like(w.H)
-    dW = torch.empty(w.W.shape, dtype=torch.float32, device=dev)
+    dW = torch.empty(W_head.shape, dtype=torch.float32, device=dev)
     # extra HBM = everything allocated beyond inputs and gradients (the workspace)
     torch.cuda.synchronize()
     base_mem = torch.cuda.memory_allocated(dev)
     torch.cuda.reset_peak_memory_stats(dev)
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
+    if vocab:
+        shard = vpm.ShardPass(w.H, W_head, v_begin=v0, V_total=w.V, dW=dW, workspace=workspace,
+                              **kw)
+        comm = vpm.TorchComm()
 
     if args.entry == "split":
         ws_split = max(ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD),
@@ -239,6 +263,9 @@ def gpu_arm(args):
         g_one = torch.ones((), dtype=torch.float32, device=dev)
 
     def step():
+        if shard is not None:
+            vpm.run_pass(shard, comm)
+            return
         if args.entry == "split":
             _lib.check(_lib.kl_fwd(prob, workspace.data_ptr(), ws_bytes, loss.data_ptr(),
                                    lse_s.data_ptr(), None if lse_t is None else lse_t.data_ptr(),
@@ -290,7 +317,7 @@ def gpu_arm(args):
     # step i's kernels run, and every step's loss is read back to pinned host
     # memory.  All copies of the K steps lie inside the timed region.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not vocab:
         from chunked_kl_loss_tma_b200.staging import HostStager
 
         names = ["H", "mask", "topk_idx", "topk_logit", "teacher_lse", "Ht"]
@@ -340,7 +367,7 @@ def gpu_arm(args):
 
     peaks, peak_src = measured_peaks()
     N, d, V = args.N, w.d, w.V
-    tok_s = ws * N * args.steps / (ms / 1e3)
+    tok_s = (1 if vocab else ws) * N * args.steps / (ms / 1e3)
     dom = max(prof, key=lambda p: p["total_ms"]) if prof else None
     roof = None
     if dom is not None:
@@ -371,14 +398,18 @@ def gpu_arm(args):
     line = {
         "metric": METRIC, "value": round(tok_s, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if vocab else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init heads and teacher cache)",
         "config": {"workload": WORKLOADS[args.workload], "N_per_gpu": N, "d": d, "V": V,
                    "K": w.K or None, "d_t": w.d_t if w.mode == "hidden" else None, "T": w.T,
                    "masked_tokens": int((w.mask == 0).sum().item()) if w.mask is not None else 0,
                    "chunk_tokens": args.chunk or min(4096, N),
                    "l2": "inputs larger than L2 (W 0.79 GB, logit chunk 1.05 GB); no flush",
-                   "parallelism": f"weak-scaling token shards x{ws}, no data-path collective"},
+                   "parallelism": (f"vocabulary-parallel head shards x{ws}: all-gather of row "
+                                   "statistics per chunk, all-reduce of fp32 dH"
+                                   if vocab else
+                                   f"weak-scaling token shards x{ws}, no data-path collective")},
         "entry": "kl_fwd_bwd" if args.entry == "fused" else "kl_fwd + kl_bwd (recompute)",
         "tensor_tflops_step": round(step_tflops, 1),
         "tensor_frac_step": round(step_tflops / peaks.get("bf16_tflops_sustained", 1400.0), 4),
@@ -396,6 +427,10 @@ def gpu_arm(args):
     if args.reverse_weight > 0:
         line["metric"] += f" [reverse KL weight {args.reverse_weight}]"
         line["config"]["reverse_weight"] = args.reverse_weight
+    if vocab:
+        line["metric"] += " [vocabulary-parallel]"
+        line["config"]["N_per_gpu"] = None
+        line["config"]["N"] = N
     if args.entry == "split":
         line["metric"] += " [kl_fwd + kl_bwd]"
         # backward recomputes the student (and teacher) logits once more

@@ -132,31 +132,40 @@ class ShardPass:
 
 
 class TorchComm:
-    """The pass's collectives over a torch.distributed process group (NCCL for
-    device tensors; gloo works for host tensors)."""
+    """The pass's collectives over a torch.distributed process group: NCCL on
+    device tensors; with another backend (gloo) device tensors go through host
+    copies and the reductions run synchronously."""
 
     def __init__(self, group=None):
         self.group = group
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.nccl = self.world > 1 and dist.get_backend(group) == "nccl"
 
     def all_gather_rows(self, t):
         """[rows, k] from every rank -> [world * rows, k], rank-major."""
         if self.world == 1:
             return t
-        out = torch.empty((self.world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype,
-                          device=t.device)
-        if dist.get_backend(self.group) == "nccl":
+        if self.nccl:
+            out = torch.empty((self.world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype,
+                              device=t.device)
             dist.all_gather_into_tensor(out, t.contiguous(), group=self.group)
-        else:
-            parts = list(out.split(t.shape[0]))
-            dist.all_gather(parts, t.contiguous(), group=self.group)
-        return out
+            return out
+        h = t.detach().to("cpu").contiguous()
+        out = torch.empty((self.world * h.shape[0],) + tuple(h.shape[1:]), dtype=h.dtype)
+        dist.all_gather(list(out.split(h.shape[0])), h, group=self.group)
+        return out.to(t.device)
 
     def all_reduce_sum(self, t, async_op=False):
+        """In-place sum over ranks; a handle to wait on when async_op and NCCL."""
         if self.world == 1:
             return None
-        return dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group, async_op=async_op)
+        if self.nccl:
+            return dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group, async_op=async_op)
+        h = t.detach().to("cpu")
+        dist.all_reduce(h, op=dist.ReduceOp.SUM, group=self.group)
+        t.copy_(h)
+        return None
 
 
 def run_pass(shard, comm, grad_loss=1.0):
@@ -178,7 +187,7 @@ def run_pass(shard, comm, grad_loss=1.0):
     if shard.row_loss is not None:
         comm.all_reduce_sum(shard.row_loss)
     return dict(loss=shard.loss, row_loss=shard.row_loss, lse_s=shard.lse_s,
-                dH=shard.cast_dH(), dW=shard.dW)
+                dH=shard.cast_dH(), dW=shard.dW, workspace=shard.ws)
 
 
 def vp_kl_fwd_bwd(H, W_shard, *, v_begin, V_total, group=None, grad_loss=1.0, **kw):

@@ -171,3 +171,70 @@ def test_accumulate_dW_and_empty_problem():
                      teacher_lse=w.teacher_lse[:0], T=w.T)
     assert float(out["loss"]) == 0.0 and out["dH"].shape == (0, w.d)
     assert torch.count_nonzero(out["dW"]) == 0
+
+
+def _free_port():
+    import socket
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _two_rank_worker(rank, world, port, q):
+    import os
+
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    # host-side gloo collectives: both ranks' kernels share one GPU and never
+    # wait on each other inside a kernel
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        torch.cuda.set_device(0)
+        w = _topk(seed=39)
+        v0, v1 = vp.vocab_shard(w.V, world, rank)
+        out = vp.vp_kl_fwd_bwd(w.H, w.W[v0:v1], v_begin=v0, V_total=w.V, grad_loss=1.2,
+                               want_row_loss=True, want_lse=True, **_kw(w, chunk=128))
+        torch.cuda.synchronize()
+        ref = _oracle(w, grad_loss=1.2)
+        dW = out["dW"].double().cpu().numpy()
+        res = dict(rank=rank, status=ops.status(out["workspace"]),
+                   loss=float(out["loss"]), ref_loss=ref["loss"],
+                   # row losses: |got - ref| / (5e-3 |ref| + 2e-4) <= 1, as the other tests
+                   row=float(np.max(np.abs(out["row_loss"].cpu().numpy() - ref["row_loss"]) /
+                                    (5e-3 * np.abs(ref["row_loss"]) + 2e-4))),
+                   lse=float(np.max(np.abs(out["lse_s"].cpu().numpy() - ref["lse_s"]))),
+                   dH=float(np.max(np.abs(out["dH"].double().cpu().numpy() - ref["dH"]))),
+                   dH_scale=float(np.max(np.abs(ref["dH"]))),
+                   dW=float(np.max(np.abs(dW - ref["dW"][v0:v1]))),
+                   dW_scale=float(np.max(np.abs(ref["dW"]))))
+        q.put(res)
+    except Exception as e:  # report instead of leaving the parent waiting
+        q.put(dict(rank=rank, error=repr(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_processes_over_gloo_on_one_gpu():
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_two_rank_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in res:
+        assert "error" not in r, r
+        assert r["status"] == 0, r
+        assert abs(r["loss"] - r["ref_loss"]) <= LOSS_RTOL * abs(r["ref_loss"]), r
+        assert r["row"] <= 1.0 and r["lse"] <= 1e-4, r
+        assert r["dH"] <= GRAD_FRAC * r["dH_scale"], r
+        assert r["dW"] <= GRAD_FRAC * r["dW_scale"], r
