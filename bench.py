@@ -297,15 +297,20 @@ def gpu_arm(args):
     launches0 = _lib.kl_launch_count()
     _lib.kl_profile_begin()
     barrier()
+    # one event after every step as well: the per-step distribution (median)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e0.record()
-    for _ in range(args.steps):
+    for i in range(args.steps):
         step()
+        marks[i].record()
     e1.record()
     barrier()
     prof = _lib.kl_profile_end()
     launches = _lib.kl_launch_count() - launches0
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    per_step = sorted([e0.elapsed_time(marks[0])] +
+                      [marks[i - 1].elapsed_time(marks[i]) for i in range(1, args.steps)])
     peak_extra = torch.cuda.max_memory_allocated(dev) - base_mem
     if ws > 1:
         ms = max_over_ranks(ms)
@@ -411,6 +416,9 @@ def gpu_arm(args):
                                    if vocab else
                                    f"weak-scaling token shards x{ws}, no data-path collective")},
         "entry": "kl_fwd_bwd" if args.entry == "fused" else "kl_fwd + kl_bwd (recompute)",
+        "step_ms_median": round(per_step[len(per_step) // 2], 4),
+        "step_ms_p10_p90": [round(per_step[len(per_step) // 10], 4),
+                            round(per_step[(9 * len(per_step)) // 10], 4)],
         "tensor_tflops_step": round(step_tflops, 1),
         "tensor_frac_step": round(step_tflops / peaks.get("bf16_tflops_sustained", 1400.0), 4),
         "tensor_frac_step_burst_peak": round(step_tflops / peaks.get("bf16_tflops", 1590.0), 4),

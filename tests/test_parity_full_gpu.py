@@ -204,3 +204,31 @@ def test_scaling_sweep_rows_and_flat_memory(N):
     _check_rows(w, out, rows, N)
     _loss_is_mean_of_rows(out, N)
     _identities(w, out)
+
+
+@pytest.mark.parametrize("cfg,P", [("offline_topk", 8), ("full_vocab", 4)])
+def test_vocabulary_parallel_full_size(cfg, P):
+    """The head split over P vocabulary shards (emulated one after another on
+    one GPU, each shard with its own workspace and the bench's chunking): the
+    oracle's sampled rows, the identities, and agreement with the whole-head
+    fused call."""
+    from chunked_kl_loss_tma_b200 import vocab_parallel as vp
+
+    w = wl.offline_topk(device="cuda", seed=7) if cfg == "offline_topk" else \
+        wl.full_vocab(device="cuda", seed=8)
+    kw = _kw(w)
+    Wt = kw.pop("Wt", None)
+    out = vp.emulate(w.H, w.W, P, Wt=Wt, want_row_loss=True, want_lse=True, **kw)
+    assert all(ops.status(ws) == 0 for ws in out["workspaces"])
+    del out["workspaces"]
+    rows = _rows(w.N, None, n_random=12, seed=P)
+    ref = _check_rows(w, out, rows, w.N)
+    r = torch.as_tensor(rows, device="cuda")
+    np.testing.assert_allclose(out["lse_s"][r].double().cpu().numpy(), ref["lse_s"], rtol=1e-5)
+    _loss_is_mean_of_rows(out, w.N)
+    _identities(w, out)
+    whole = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w))
+    assert abs(out["loss"].item() - whole["loss"].item()) <= 1e-5 * abs(whole["loss"].item())
+    for k in ("dH", "dW"):
+        a, c = out[k].double(), whole[k].double()
+        assert (a - c).abs().max().item() <= 1e-2 * c.abs().max().item(), k
