@@ -351,3 +351,33 @@ def test_split_backward_accumulates_into_dW():
     b = ops.kl_bwd(w.H, w.W, f["lse_s"], dW=base.clone(), accumulate_dW=True, **kw)
     ref = _oracle(w)
     _check_grad(b["dW"] - base, ref["dW"], "accumulated dW (split)")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("N,d,V,K", [(1, 8, 1, 1), (3, 8, 7, 2), (5, 16, 9, 9), (2, 8, 300, 1)])
+def test_smallest_shapes(dtype, N, d, V, K):
+    """One-row, one-class and sub-vector vocabularies (V < 8 pads the logit
+    rows), the narrowest width d = 8 and a single cached entry, both teacher
+    modes.  With V = 1 both distributions are a point mass: loss 0 up to
+    rounding."""
+    w = wl.make_topk("tiny_shapes", N=N, d=d, V=V, K=K, d_t=8, T=1.1, dtype=dtype,
+                     w_std=0.3, tw_std=0.3, seed=50 + V).to("cuda")
+    for partial in (True, False):
+        kw = _kw(w)
+        if not partial:
+            kw["teacher_lse"] = None
+        out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
+        assert ops.status(out["workspace"]) == 0
+        ref = _oracle(w, teacher_lse=kw["teacher_lse"])
+        assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-5
+        for k in ("dH", "dW"):
+            got = out[k].double().cpu().numpy()
+            assert np.max(np.abs(got - ref[k])) <= GRAD_FRAC * np.max(np.abs(ref[k])) + 1e-6, k
+    h = wl.make_hidden("tiny_shapes_h", N=N, d=d, d_t=8, V=V, T=1.1, dtype=dtype, w_std=0.3,
+                       tw_std=0.3, seed=60 + V).to("cuda")
+    out = ops.kl_fwd_bwd(h.H, h.W, want_row_loss=True, **_kw(h))
+    ref = _oracle(h)
+    assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-5
+    for k in ("dH", "dW"):
+        got = out[k].double().cpu().numpy()
+        assert np.max(np.abs(got - ref[k])) <= GRAD_FRAC * np.max(np.abs(ref[k])) + 1e-6, k
