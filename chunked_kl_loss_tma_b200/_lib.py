@@ -28,8 +28,8 @@ KL_NOALLOC_SCRATCH_BYTES = 16 << 20
 # Every symbol declared in include/chunked_kl.h.
 EXPORTS = ("kl_workspace_bytes", "kl_fwd", "kl_bwd", "kl_fwd_bwd", "kl_status",
            "kl_status_string", "kl_launch_count", "kl_profile_begin", "kl_profile_end",
-           "kl_fwd_noalloc", "kl_vp_num_chunks", "kl_vp_fwd_chunk", "kl_vp_bwd_chunk",
-           "kl_cast_f32")
+           "kl_fwd_noalloc", "kl_vp_num_chunks", "kl_vp_fwd_chunk", "kl_vp_mid_chunk",
+           "kl_vp_bwd_chunk", "kl_cast_f32")
 
 
 class KLProblem(ctypes.Structure):
@@ -88,7 +88,10 @@ def lib():
     L.kl_vp_num_chunks.restype = i64
     L.kl_vp_fwd_chunk.argtypes = [P, i64, vp, sz, vp, vp]
     L.kl_vp_fwd_chunk.restype = i32
-    L.kl_vp_bwd_chunk.argtypes = [P, i64, vp, sz, vp, i32, i32, f32, vp, vp, vp, vp, vp, i32, vp]
+    L.kl_vp_mid_chunk.argtypes = [P, i64, vp, sz, vp, i32, i32, vp, vp]
+    L.kl_vp_mid_chunk.restype = i32
+    L.kl_vp_bwd_chunk.argtypes = [P, i64, vp, sz, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, i32,
+                                  vp]
     L.kl_vp_bwd_chunk.restype = i32
     L.kl_cast_f32.argtypes = [vp, vp, i64, i32, vp]
     L.kl_cast_f32.restype = i32
@@ -150,11 +153,16 @@ def kl_vp_fwd_chunk(prob, chunk, ws, ws_bytes, row_stats, stream):
     return lib().kl_vp_fwd_chunk(ctypes.byref(prob), int(chunk), ws, ws_bytes, row_stats, stream)
 
 
-def kl_vp_bwd_chunk(prob, chunk, ws, ws_bytes, row_stats_all, P, rank, grad_loss, loss, lse_s,
-                    row_loss, dH_part, dW, accumulate_dW, stream):
+def kl_vp_mid_chunk(prob, chunk, ws, ws_bytes, row_stats_all, P, rank, sums, stream):
+    return lib().kl_vp_mid_chunk(ctypes.byref(prob), int(chunk), ws, ws_bytes, row_stats_all,
+                                 int(P), int(rank), sums, stream)
+
+
+def kl_vp_bwd_chunk(prob, chunk, ws, ws_bytes, row_stats_all, sums_all, P, rank, grad_loss, loss,
+                    lse_s, row_loss, dH_part, dW, accumulate_dW, stream):
     return lib().kl_vp_bwd_chunk(ctypes.byref(prob), int(chunk), ws, ws_bytes, row_stats_all,
-                                 int(P), int(rank), float(grad_loss), loss, lse_s, row_loss,
-                                 dH_part, dW, int(accumulate_dW), stream)
+                                 sums_all, int(P), int(rank), float(grad_loss), loss, lse_s,
+                                 row_loss, dH_part, dW, int(accumulate_dW), stream)
 
 
 def kl_cast_f32(src, dst, n, dtype, stream):

@@ -732,7 +732,9 @@ template <typename Elem>
 int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
                         const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
                         float* row_loss, int write_grad, const float4* part_s,
-                        const float4* part_t, int add_lse = 1) {
+                        const float4* part_t, int add_lse = 1, int phase = kDlfBoth,
+                        float* sums_out = nullptr, const float* sums_all = nullptr, int P = 1,
+                        int rank = 0) {
   const kl_problem* p = c.p;
   LaunchScope ls("dlogits_full", c.st, 0,
                  ((write_grad ? 3.0 : 2.0) + (p->reverse_weight > 0.f && write_grad ? 2.0 : 0.0)) *
@@ -741,7 +743,8 @@ int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
       S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
       p->T_row ? p->T_row + c0 : nullptr, row_loss ? row_loss + c0 : nullptr, write_grad,
-      p->reverse_weight, part_s, part_t, c.pl.tiles_v, add_lse);
+      p->reverse_weight, part_s, part_t, c.pl.tiles_v, add_lse, phase, sums_out, sums_all, P,
+      rank, static_cast<int>(Cn));
   return KL_LAUNCHED();
 }
 
@@ -928,10 +931,43 @@ int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
   return launch_row_stats(c, pt, Cn, stats, 1, false);
 }
 
+// Merge the P shards' row statistics of chunk k: whole-vocabulary lse_s (and
+// lse_t) into the workspace (and lse_user), and the top-K row-loss share.
+int launch_vp_merge(Ctx& c, int64_t c0, int64_t Cn, const float* stats_all, int P, int rank,
+                    float* lse_user, float* rl) {
+  const kl_problem* p = c.p;
+  float* lse_s = reinterpret_cast<float*>(c.ws + c.pl.off_lse_s);
+  float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
+  LaunchScope ls("vp_merge", c.st, 0, static_cast<double>(Cn) * (8.0 * P + 12));
+  vp_merge_kernel<<<static_cast<unsigned>(cdiv(Cn, 128)), 128, 0, c.st>>>(
+      stats_all, P, static_cast<int>(Cn), c.pl.hidden ? 1 : 0, rank,
+      p->mask ? p->mask + c0 : nullptr,
+      c.pl.hidden ? nullptr : reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
+      lse_s + c0, lse_t ? lse_t + c0 : nullptr, lse_user ? lse_user + c0 : nullptr, rl + c0);
+  return KL_LAUNCHED();
+}
+
+// Teacher-hidden mode with a reverse-KL weight: this shard's sums (A, U) of
+// chunk k, written to sums_out [rows][2].
 template <typename Elem>
-int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank, float g,
-                     float* loss, float* lse_user, float* row_loss, float* dH, float* dW,
-                     int accumulate) {
+int run_vp_mid_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank,
+                     float* sums_out) {
+  int64_t c0, Cn;
+  chunk_rows(c, k, &c0, &Cn);
+  float* rl = reinterpret_cast<float*>(c.ws + c.pl.off_rl);
+  KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, nullptr, rl));
+  return launch_dlogits_full<Elem>(
+      c, reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf), reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf),
+      c0, Cn, reinterpret_cast<float*>(c.ws + c.pl.off_lse_s),
+      reinterpret_cast<float*>(c.ws + c.pl.off_lse_t), nullptr, 0.f, nullptr, 0,
+      reinterpret_cast<float4*>(c.ws + c.pl.off_ps), reinterpret_cast<float4*>(c.ws + c.pl.off_pt),
+      0, kDlfSums, sums_out, nullptr, P, rank);
+}
+
+template <typename Elem>
+int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sums_all, int P,
+                     int rank, float g, float* loss, float* lse_user, float* row_loss, float* dH,
+                     float* dW, int accumulate) {
   const kl_problem* p = c.p;
   int64_t c0, Cn;
   chunk_rows(c, k, &c0, &Cn);
@@ -940,22 +976,16 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank,
   float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
   Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
-  {
-    LaunchScope ls("vp_merge", c.st, 0, static_cast<double>(Cn) * (8.0 * P + 12));
-    vp_merge_kernel<<<static_cast<unsigned>(cdiv(Cn, 128)), 128, 0, c.st>>>(
-        stats_all, P, static_cast<int>(Cn), c.pl.hidden ? 1 : 0, rank,
-        p->mask ? p->mask + c0 : nullptr,
-        c.pl.hidden ? nullptr : reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo),
-        lse_s + c0, lse_t ? lse_t + c0 : nullptr, lse_user ? lse_user + c0 : nullptr, rl + c0);
-    KL_TRY(KL_LAUNCHED());
-  }
+  KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, lse_user, rl));
   if (!c.pl.hidden) {
     KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
   } else {
     Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
     float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+    const bool split = p->reverse_weight > 0.f;  // u_bar came through the second exchange
     KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1, ps, pt,
-                                     rank == 0 ? 1 : 0));
+                                     rank == 0 ? 1 : 0, split ? kDlfGrad : kDlfBoth, nullptr,
+                                     sums_all, P, rank));
   }
   KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || k > 0) ? 1 : 0, true));
   if (c0 + Cn == p->N) KL_TRY(launch_finalize(c, rl, loss));
@@ -966,7 +996,6 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank,
 int vp_begin(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes, void* stream,
              Ctx& c) {
   KL_TRY(validate(p));
-  if (p->reverse_weight != 0.f) return KL_ERR_ARG;
   if (chunk < 0 || chunk >= num_chunks(p, make_plan(p, KL_ENTRY_FWD_BWD).C)) return KL_ERR_ARG;
   return begin(p, KL_ENTRY_FWD_BWD, ws, ws_bytes, stream, c, true);
 }
@@ -1034,22 +1063,36 @@ int kl_vp_fwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_byte
                                    : run_vp_fwd_chunk<float>(c, chunk, row_stats);
 }
 
+int kl_vp_mid_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    const float* row_stats_all, int P, int rank, float* sums, void* stream) {
+  if (P < 1 || rank < 0 || rank >= P) return KL_ERR_ARG;
+  if (p != nullptr && p->teacher != KL_TEACHER_HIDDEN) return KL_ERR_ARG;
+  Ctx c;
+  KL_TRY(vp_begin(p, chunk, ws, ws_bytes, stream, c));
+  if (row_stats_all == nullptr || sums == nullptr) return KL_ERR_NULL;
+  return p->dtype == KL_DTYPE_BF16
+             ? run_vp_mid_chunk<__nv_bfloat16>(c, chunk, row_stats_all, P, rank, sums)
+             : run_vp_mid_chunk<float>(c, chunk, row_stats_all, P, rank, sums);
+}
+
 int kl_vp_bwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
-                    const float* row_stats_all, int P, int rank, float grad_loss, float* loss,
-                    float* lse_s, float* row_loss, float* dH_part, float* dW, int accumulate_dW,
-                    void* stream) {
+                    const float* row_stats_all, const float* sums_all, int P, int rank,
+                    float grad_loss, float* loss, float* lse_s, float* row_loss, float* dH_part,
+                    float* dW, int accumulate_dW, void* stream) {
   if (P < 1 || rank < 0 || rank >= P) return KL_ERR_ARG;
   Ctx c;
   KL_TRY(vp_begin(p, chunk, ws, ws_bytes, stream, c));
-  if (row_stats_all == nullptr || loss == nullptr || dH_part == nullptr || dW == nullptr)
+  if (row_stats_all == nullptr || loss == nullptr || dH_part == nullptr || dW == nullptr ||
+      (p->reverse_weight > 0.f && sums_all == nullptr))
     return KL_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(dH_part) | reinterpret_cast<uintptr_t>(dW)) & 15)
     return KL_ERR_ALIGN;
   return p->dtype == KL_DTYPE_BF16
-             ? run_vp_bwd_chunk<__nv_bfloat16>(c, chunk, row_stats_all, P, rank, grad_loss, loss,
-                                               lse_s, row_loss, dH_part, dW, accumulate_dW)
-             : run_vp_bwd_chunk<float>(c, chunk, row_stats_all, P, rank, grad_loss, loss, lse_s,
-                                       row_loss, dH_part, dW, accumulate_dW);
+             ? run_vp_bwd_chunk<__nv_bfloat16>(c, chunk, row_stats_all, sums_all, P, rank,
+                                               grad_loss, loss, lse_s, row_loss, dH_part, dW,
+                                               accumulate_dW)
+             : run_vp_bwd_chunk<float>(c, chunk, row_stats_all, sums_all, P, rank, grad_loss,
+                                       loss, lse_s, row_loss, dH_part, dW, accumulate_dW);
 }
 
 int kl_cast_f32(const float* src, void* dst, int64_t n, int dtype, void* stream) {

@@ -365,6 +365,14 @@ __device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
 //   dS = c [(1 - beta)(p_s - p_t) + beta p_s (u - u_bar)],  u = s~ - t~,
 // written in place over S in a second pass (u_bar is needed first).  With
 // beta = 0 the single pass writes dS = c (p_s - p_t).
+// phase: kDlfBoth does the above; for a vocabulary shard with beta > 0 the
+// two passes are split around an exchange: kDlfSums writes this shard's
+// (A, U) to sums_out[row] and nothing else, and kDlfGrad reads every shard's
+// (A, U) from sums_all ([P][rows][2], rank order), takes u_bar as the sum of
+// the U and runs only the second pass (the row loss from this shard's A, U).
+constexpr int kDlfBoth = 0;
+constexpr int kDlfSums = 1;
+constexpr int kDlfGrad = 2;
 template <typename Elem>
 __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict__ Tt, int64_t ld,
                                     int V, const float* __restrict__ lse_s,
@@ -375,7 +383,9 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
                                     float* __restrict__ row_loss, int write_grad, float beta,
                                     const float4* __restrict__ part_s,
                                     const float4* __restrict__ part_t, int tiles_n,
-                                    int add_lse) {
+                                    int add_lse, int phase, float* __restrict__ sums_out,
+                                    const float* __restrict__ sums_all, int P, int rank,
+                                    int rows) {
   __shared__ float2 red[32];
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
@@ -385,7 +395,7 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
   const int nvec = (V + 7) >> 3;
   const bool single = beta == 0.f;
   float A = 0.f, U = 0.f;
-  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+  for (int v = (phase == kDlfGrad ? nvec : 0) + threadIdx.x; v < nvec; v += blockDim.x) {
     float fs[8], ft[8];
     load8<Elem>(srow + v * 8, fs);
     load8<Elem>(trow + v * 8, ft);
@@ -405,8 +415,24 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
     }
     if (write_grad && single) store8<Elem>(srow + v * 8, fs);
   }
-  const float2 r = block_sum2(A, U, red);
-  const float ubar = r.y;
+  float2 r;
+  float ubar;
+  if (phase == kDlfGrad) {  // every shard's sums, merged in rank order
+    const int64_t blk = static_cast<int64_t>(rows) * 2;
+    r = make_float2(sums_all[rank * blk + 2 * row], sums_all[rank * blk + 2 * row + 1]);
+    ubar = 0.f;
+    for (int q = 0; q < P; ++q) ubar += sums_all[q * blk + 2 * row + 1];
+  } else {
+    r = block_sum2(A, U, red);
+    ubar = r.y;
+  }
+  if (phase == kDlfSums) {
+    if (threadIdx.x == 0) {
+      sums_out[2 * row] = r.x;
+      sums_out[2 * row + 1] = r.y;
+    }
+    return;
+  }
   if (write_grad && !single) {
     const float cf = coef * (1.f - beta), cr = coef * beta;
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
@@ -432,7 +458,7 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict
     // add_lse = 0: a vocabulary shard's share, the sums over its columns only
     const float dl = add_lse ? lse_s[row] - lse_t[row] : 0.f;
     const float fwd = r.x + dl;
-    const float rev = ubar - dl;
+    const float rev = r.y - dl;
     row_loss[row] = keep ? (1.f - beta) * fwd + beta * rev : 0.f;
   }
 }

@@ -14,9 +14,15 @@ token chunk suffices:
     for each chunk k:
         kl_vp_fwd_chunk   logits over the shard, row statistics  (kernels)
         all-gather        the P ranks' statistics, rank order    (NCCL)
+      [ kl_vp_mid_chunk   the shard's sums (A, U)                (kernels)
+        all-gather        the P ranks' sums                      (NCCL) ]
         kl_vp_bwd_chunk   merge, dS, this rank's dH share, own dW rows (kernels)
         all-reduce        the chunk's fp32 dH shares, async      (NCCL)
     all-reduce the loss shares; kl_cast_f32 turns the summed dH into H's dtype.
+
+The bracketed steps run in the teacher-hidden mode with a reverse-KL weight
+only: that gradient needs sum_j p_s,j (s~_j - t~_j) over the whole vocabulary
+before dS is written.
 
 The arithmetic is in the library's kernels; this module orders the calls and
 the collectives.  `emulate` runs P shards one after another on one device
@@ -90,6 +96,9 @@ class ShardPass:
         self.accumulate = bool(accumulate_dW)
         C = self.chunks[0][1] if self.chunks else 1
         self._stats = torch.empty(C, 2, dtype=torch.float32, device=dev)
+        self.two_exchanges = float(kw.get("reverse_weight", 0.0)) > 0.0
+        self._sums = torch.empty(C, 2, dtype=torch.float32, device=dev) \
+            if self.two_exchanges else None
         self._stream = torch.cuda.current_stream(dev).cuda_stream
 
     def fwd_chunk(self, k):
@@ -100,13 +109,26 @@ class ShardPass:
                                   self._stream), "kl_vp_fwd_chunk")
         return st
 
-    def bwd_chunk(self, k, stats_all, P, rank, grad_loss=1.0):
-        """Chunk k's gradients from every rank's statistics [P * rows, 2] (rank order)."""
+    def mid_chunk(self, k, stats_all, P, rank):
+        """Chunk k's sums (A, U) over the shard [rows, 2] (reverse-KL weight > 0)."""
         rows = self.chunks[k][1]
         if stats_all.shape != (P * rows, 2) or not stats_all.is_contiguous():
             raise ValueError("stats_all must be a contiguous [P * rows, 2] tensor")
+        out = self._sums[:rows]
+        L.check(L.kl_vp_mid_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel(),
+                                  stats_all.data_ptr(), P, rank, out.data_ptr(), self._stream),
+                "kl_vp_mid_chunk")
+        return out
+
+    def bwd_chunk(self, k, stats_all, P, rank, grad_loss=1.0, sums_all=None):
+        """Chunk k's gradients from every rank's statistics [P * rows, 2] (rank order)
+        and, with a reverse-KL weight, every rank's sums [P * rows, 2]."""
+        rows = self.chunks[k][1]
+        for t in (stats_all,) + ((sums_all,) if self.two_exchanges else ()):
+            if t is None or t.shape != (P * rows, 2) or not t.is_contiguous():
+                raise ValueError("statistics must be contiguous [P * rows, 2] tensors")
         L.check(L.kl_vp_bwd_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel(),
-                                  stats_all.data_ptr(), P, rank, grad_loss,
+                                  stats_all.data_ptr(), ops._ptr(sums_all), P, rank, grad_loss,
                                   self.loss.data_ptr(), ops._ptr(self.lse_s),
                                   ops._ptr(self.row_loss), self.dH32.data_ptr(),
                                   self.dW.data_ptr(), self.accumulate, self._stream),
@@ -176,8 +198,11 @@ def run_pass(shard, comm, grad_loss=1.0):
     if not shard.chunks:
         shard.empty_pass()
     for k in range(len(shard.chunks)):
-        st = shard.fwd_chunk(k)
-        shard.bwd_chunk(k, comm.all_gather_rows(st), comm.world, comm.rank, grad_loss)
+        st_all = comm.all_gather_rows(shard.fwd_chunk(k))
+        sums_all = None
+        if shard.two_exchanges:
+            sums_all = comm.all_gather_rows(shard.mid_chunk(k, st_all, comm.world, comm.rank))
+        shard.bwd_chunk(k, st_all, comm.world, comm.rank, grad_loss, sums_all)
         h = comm.all_reduce_sum(shard.dH_rows(k), async_op=True)
         if h is not None:
             pending.append(h)
@@ -218,8 +243,11 @@ def emulate(H, W, P, *, shards=None, grad_loss=1.0, Wt=None, **kw):
             s.empty_pass()
     for k in range(len(passes[0].chunks)):
         stats = torch.cat([s.fwd_chunk(k) for s in passes])
+        sums = None
+        if passes[0].two_exchanges:
+            sums = torch.cat([s.mid_chunk(k, stats, len(passes), r) for r, s in enumerate(passes)])
         for r, s in enumerate(passes):
-            s.bwd_chunk(k, stats, len(passes), r, grad_loss)
+            s.bwd_chunk(k, stats, len(passes), r, grad_loss, sums)
     loss = sum(s.loss for s in passes)
     row_loss = (sum(s.row_loss for s in passes) if passes[0].row_loss is not None else None)
     dH32 = passes[0].dH32.clone()

@@ -210,7 +210,10 @@ int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_lo
  *   1. kl_vp_fwd_chunk  -> row_stats [rows_k][2] of this shard
  *   2. the caller gathers all ranks' row_stats, rank-major: [P][rows_k][2]
  *      (e.g. an NCCL all-gather; 8 bytes per row per rank)
- *   3. kl_vp_bwd_chunk  -> this rank's share of the row losses and of dH
+ *   (teacher-hidden mode with reverse_weight > 0 only:
+ *   3a. kl_vp_mid_chunk -> sums [rows_k][2] of this shard, (A, U) below
+ *   3b. the caller gathers all ranks' sums, rank-major: [P][rows_k][2])
+ *   4. kl_vp_bwd_chunk  -> this rank's share of the row losses and of dH
  *      (fp32, rows of chunk k), and dW rows of its own shard
  *
  * then sums over ranks (e.g. an NCCL all-reduce) the fp32 dH partials, the
@@ -218,11 +221,13 @@ int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_lo
  * over ranks is the result.  kl_cast_f32 turns the summed fp32 dH into H's
  * dtype.  rows_k = min(C, N - k C) with C = chunk_tokens (default 4096).
  * Chunk 0 starts a pass (it resets the status word and prepares the heads);
- * the workspace carries the chunk's logits from step 1 to step 3, so no other
- * call may use it in between.  Requires reverse_weight = 0 (the reverse-KL
- * gradient needs a second per-row exchange; not provided): KL_ERR_ARG.
- * Errors as kl_fwd_bwd, plus KL_ERR_ARG for v_begin < 0, v_begin + V > V_total,
- * chunk outside [0, kl_vp_num_chunks()), P < 1 or rank outside [0, P). */
+ * the workspace carries the chunk's logits from step 1 to step 4, so no other
+ * call may use it in between.  The reverse-KL gradient needs
+ * u_bar = sum_j p_s,j (s~_j - t~_j) over the whole vocabulary before dS can be
+ * written, hence the second exchange (A = sum_j p_t,j (t~_j - s~_j) travels with
+ * it for the row loss).  Errors as kl_fwd_bwd, plus KL_ERR_ARG for v_begin < 0,
+ * v_begin + V > V_total, chunk outside [0, kl_vp_num_chunks()), P < 1 or rank
+ * outside [0, P). */
 
 /* Number of token chunks of the pass (0 when N = 0), or -1 if p is invalid. */
 int64_t kl_vp_num_chunks(const kl_problem* p);
@@ -234,18 +239,27 @@ int64_t kl_vp_num_chunks(const kl_problem* p);
 int kl_vp_fwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
                     float* row_stats, void* stream);
 
-/* Step 3 for chunk k.  row_stats_all: [P][rows_k][2], every rank's step-1
- * output in rank order.  Writes lse_s [N] rows of the chunk (whole-vocabulary
- * student lse; may be NULL), row_loss [N] rows of the chunk (this rank's share;
- * may be NULL), dH_part [N, d] fp32 rows of the chunk (this rank's share,
- * dS_shard . W_shard), and dW [V, d] fp32 (this shard's rows; overwritten at
- * chunk 0 unless accumulate_dW, accumulated otherwise).  After the last chunk
- * it writes loss (device scalar, this rank's share of the mean).  grad_loss is
- * the incoming gradient g.  Tensor work: 4 rows_k d V. */
+/* Step 3a for chunk k (KL_TEACHER_HIDDEN, else KL_ERR_ARG): from every rank's
+ * step-1 output row_stats_all [P][rows_k][2], this shard's sums over its
+ * columns, sums[i] = (A_r, U_r) with A_r = sum p_t (t~ - s~) and
+ * U_r = sum p_s (s~ - t~), p_s and p_t the whole-vocabulary softmaxes. */
+int kl_vp_mid_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
+                    const float* row_stats_all, int P, int rank, float* sums, void* stream);
+
+/* Step 4 for chunk k.  row_stats_all: [P][rows_k][2], every rank's step-1
+ * output in rank order; sums_all: [P][rows_k][2], every rank's step-3a output
+ * (required when reverse_weight > 0, ignored otherwise).  Writes lse_s [N] rows
+ * of the chunk (whole-vocabulary student lse; may be NULL), row_loss [N] rows
+ * of the chunk (this rank's share; may be NULL), dH_part [N, d] fp32 rows of
+ * the chunk (this rank's share, dS_shard . W_shard), and dW [V, d] fp32 (this
+ * shard's rows; overwritten at chunk 0 unless accumulate_dW, accumulated
+ * otherwise).  After the last chunk it writes loss (device scalar, this rank's
+ * share of the mean).  grad_loss is the incoming gradient g.  Tensor work:
+ * 4 rows_k d V. */
 int kl_vp_bwd_chunk(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes,
-                    const float* row_stats_all, int P, int rank, float grad_loss, float* loss,
-                    float* lse_s, float* row_loss, float* dH_part, float* dW, int accumulate_dW,
-                    void* stream);
+                    const float* row_stats_all, const float* sums_all, int P, int rank,
+                    float grad_loss, float* loss, float* lse_s, float* row_loss, float* dH_part,
+                    float* dW, int accumulate_dW, void* stream);
 
 /* dst[i] = src[i] converted to dtype (KL_DTYPE_BF16: round to nearest even;
  * KL_DTYPE_F32: copy), i < n; n a multiple of 4, both 16-byte aligned. */

@@ -120,13 +120,16 @@ def test_vocab_parallel_host_checks(lib):
     # chunk index, rank and reverse weight are checked before the device
     assert L.kl_vp_fwd_chunk(p, 4, 256, 1 << 40, 256, None) == 10
     assert L.kl_vp_fwd_chunk(p, -1, 256, 1 << 40, 256, None) == 10
-    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, 2, 2, 1.0, 256, None, None, 256, 256, 0,
-                             None) == 10
-    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, 0, 0, 1.0, 256, None, None, 256, 256, 0,
-                             None) == 10
+    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, None, 2, 2, 1.0, 256, None, None, 256,
+                             256, 0, None) == 10
+    assert L.kl_vp_bwd_chunk(p, 0, 256, 1 << 40, 256, None, 0, 0, 1.0, 256, None, None, 256,
+                             256, 0, None) == 10
+    # the middle phase exists for the teacher-hidden mode only
+    assert L.kl_vp_mid_chunk(p, 0, 256, 1 << 40, 256, 2, 0, 256, None) == 10
     q = _problem(teacher=1, d_t=4096, K=0, V=4096, V_total=128256, reverse_weight=0.5)
     q.H = q.W = q.Ht = q.Wt = 256
-    assert L.kl_vp_fwd_chunk(q, 0, 256, 1 << 40, 256, None) == 10
+    assert L.kl_vp_mid_chunk(q, 0, 256, 1 << 40, 256, 0, 0, 256, None) == 10   # P < 1
+    assert L.kl_vp_mid_chunk(q, 9, 256, 1 << 40, 256, 2, 1, 256, None) == 10   # no chunk 9
 
 
 def test_cast_host_checks(lib):

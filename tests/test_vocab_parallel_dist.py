@@ -66,6 +66,8 @@ class NumpyShard:
         self.lse_s = torch.zeros(N, dtype=torch.float64)
         self.dH32 = torch.zeros(N, d, dtype=torch.float64)
         self.dW = torch.zeros(v1 - v0, d, dtype=torch.float64)
+        self.two_exchanges = False  # top-K mode: one exchange per chunk
+        self.ws = None
 
     def _local(self, rows):
         """Cached entries of these rows inside the shard: (row, local col, q)."""
@@ -80,7 +82,7 @@ class NumpyShard:
         cross = np.bincount(r, weights=q * self._s[r, c], minlength=n)
         return torch.tensor(np.stack([_lse(self._s, 1), cross], 1))
 
-    def bwd_chunk(self, k, stats_all, P, rank, grad_loss=1.0):
+    def bwd_chunk(self, k, stats_all, P, rank, grad_loss=1.0, sums_all=None):
         c0, n = self.chunks[k]
         rows = slice(c0, c0 + n)
         st = stats_all.numpy().reshape(P, n, 2)
@@ -153,6 +155,8 @@ def _worker(rank, world, port, q):
                float(np.max(np.abs(out["dH"].numpy() - ref["dH"]))),
                float(np.max(np.abs(out["dW"].numpy() - ref["dW"][v0:v1]))),
                float(np.max(np.abs(ref["dH"])))))
+    except Exception as e:  # report instead of leaving the parent waiting
+        q.put((rank, repr(e)))
     finally:
         dist.destroy_process_group()
 
@@ -168,6 +172,8 @@ def test_two_rank_vocabulary_parallel_pass_matches_whole_head_oracle():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
+    for r in res:
+        assert len(r) == 7, r
     for rank, dloss, drow, dlse, ddH, ddW, scale in res:
         assert scale > 1e-3
         assert abs(dloss) < 1e-12 and drow < 1e-12 and dlse < 1e-12, rank

@@ -106,6 +106,29 @@ def test_hidden_shards_match_oracle(dtype):
     _check_all(out, _oracle(w))
 
 
+@pytest.mark.parametrize("beta", [0.35, 1.0])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_reverse_kl_mixing_shards_match_oracle(beta, dtype):
+    """Reverse-KL weight > 0: the second exchange (every shard's sums A, U)
+    gives u_bar over the whole vocabulary before dS is written."""
+    w = _hidden(dtype=dtype, seed=34)
+    kw = dict(_kw(w, chunk=96), reverse_weight=beta)
+    Wt = kw.pop("Wt")
+    out = vp.emulate(w.H, w.W, 3, shards=[(0, 1024), (1024, 1030), (1030, 3001)], Wt=Wt,
+                     grad_loss=1.3, want_row_loss=True, want_lse=True, **kw)
+    _check_all(out, _oracle(w, reverse_weight=beta, grad_loss=1.3))
+
+
+def test_reverse_kl_single_shard_is_the_fused_call_bit_for_bit():
+    w = _hidden(seed=36)
+    kw = dict(_kw(w, chunk=128), reverse_weight=0.5)
+    ref = ops.kl_fwd_bwd(w.H, w.W, grad_loss=0.7, want_row_loss=True, **kw)
+    Wt = kw.pop("Wt")
+    out = vp.emulate(w.H, w.W, 1, Wt=Wt, grad_loss=0.7, want_row_loss=True, **kw)
+    for k in ("loss", "row_loss", "dH", "dW"):
+        assert torch.equal(out[k], ref[k]), k
+
+
 def test_per_token_temperature_shards():
     g = torch.Generator().manual_seed(5)
     Tr = (0.5 + 2.5 * torch.rand(300, generator=g)).to(torch.float32)
