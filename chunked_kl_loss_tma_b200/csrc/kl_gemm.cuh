@@ -381,7 +381,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Each warp stages its 32 rows x 32 columns of output in shared memory
     // (two buffers, swizzled to match the output map) and one lane issues a TMA
     // bulk store -- an fp32 add-reduction into global memory when accumulating.
-    const int r = warp * 32 + lane;  // accumulator row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     uint8_t* stg = staging + warp * 2 * kStageOutBytes;
     const uint64_t out_policy = l2_policy_evict_first();
