@@ -226,6 +226,13 @@ int choose_ksplit(int64_t tiles, int64_t num_kb, int64_t units) {
   return best;
 }
 
+// dH (bf16) runs on wide 256 x 512 pair tiles: its work units are long (a
+// K-part of the vocabulary), so the single accumulator's unhidden epilogue
+// costs little, and sharing each A stage between two N halves cuts the operand
+// bytes a CTA pulls from L2 by a quarter.
+constexpr int kDhWide = 1;
+constexpr int kDhTileN = kDhWide ? 2 * kBN : kBN;
+
 // CTA pairs available for one contraction (the workspace plan must not depend
 // on the device, so this is the B200's 148 SMs / 2).
 int64_t max_units_hint() { return 74; }
@@ -312,7 +319,7 @@ Plan make_plan(const kl_problem* p, int entry) {
   }
   if (entry != KL_ENTRY_BWD) pl.off_rl = take(nrow);
   if (pl.eb == 2 && entry != KL_ENTRY_FWD) {
-    pl.ksplit_dh = choose_ksplit(cdiv(pl.C, 2 * kBM) * cdiv(p->d, kBN), cdiv(p->V, 64),
+    pl.ksplit_dh = choose_ksplit(cdiv(pl.C, 2 * kBM) * cdiv(p->d, kDhTileN), cdiv(p->V, 64),
                                  max_units_hint());
     if (pl.ksplit_dh > 1)
       pl.off_dhp = take(static_cast<size_t>(pl.ksplit_dh) * cdiv(pl.C, 2 * kBM) * 2 * kBM *
@@ -335,10 +342,10 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR>;
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -578,7 +585,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       return KL_ERR_CUDA;
     GemmParams gp{};
     gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
-    gp.tiles_n = static_cast<int>(cdiv(d, kBN));
+    gp.tiles_n = static_cast<int>(cdiv(d, kDhTileN));
     gp.num_kb = static_cast<int>(cdiv(p->V, kBKe));
     gp.m_fastest = 1;
     gp.rows_valid = static_cast<int>(Cn);
@@ -599,7 +606,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
       LaunchScope ls("splitk_reduce", c.st, 0,
                      (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
@@ -616,14 +623,14 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
                         d * sizeof(Elem)))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
                                                     2.0 * Cn * p->V * d)));
     }
   }

@@ -191,16 +191,26 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR>
+// WIDE = 1 (2-CTA pairs, store / accumulate epilogues): each work unit is a
+// 256 x 512 output tile computed as two N = 256 MMAs per K step that share the
+// A stage, so a CTA pulls 25% fewer operand bytes from L2 per MMA.  Both halves
+// fill all 512 TMEM columns, so there is a single accumulator: the next unit's
+// MMAs wait for the epilogue (worth it where units are long, as in dH).
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
+                "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
   constexpr int kCtas = PAIR ? 2 : 1;
-  constexpr int kNS = PAIR ? kStagesPair : kStages;   // ring depth
-  constexpr int kBRows = kBN / kCtas;                 // B rows staged by this CTA
+  constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
+  constexpr int kTileN = kBN * kHalves;               // output columns per unit
+  constexpr int kAccBufs = WIDE ? 1 : 2;              // accumulators in TMEM
+  constexpr int kBRows = kBN / kCtas;                 // B rows per half staged by this CTA
   constexpr int kBBytes = kBRows * kRowBytes;
-  constexpr int kSBytes = kATileBytes + kBBytes;      // this CTA's stage bytes
+  constexpr int kSBytes = kATileBytes + kHalves * kBBytes;  // this CTA's stage bytes
+  constexpr int kNS = PAIR ? (WIDE ? kRingBytes / kSBytes : kStagesPair) : kStages;  // ring
   constexpr int kEB = ElemTraits<Elem>::kBytes;
   constexpr int kBKe = kRowBytes / kEB;       // K elements per stage (64 / 32)
   constexpr int kUmmaK = 32 / kEB;            // K per MMA instruction (16 / 8)
@@ -273,7 +283,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int tm, tn;
         tile_coords(ur.tile, p, tm, tn);
         const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;  // this CTA's A rows
-        const int n0 = tn * kBN + static_cast<int>(rank) * kBRows;        // this CTA's B rows
+        const int n0 = tn * kTileN + static_cast<int>(rank) * kBRows;     // this CTA's B rows
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           const uint32_t s = issued % kNS;
           const uint32_t ph = (issued / kNS) & 1u;
@@ -294,11 +304,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             else tma_load_2d(&tmA, &full_bar[s], dst, x, y);
           }
 #pragma unroll
-          for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
-            void* dst = b_s + sl * kSlabBytes;
-            const int x = B_MN ? n0 + sl * kMNe : k0, y = B_MN ? k0 : n0;
-            if (PAIR) tma_load_2d_pair(&tmB, fb, dst, x, y);
-            else tma_load_2d(&tmB, &full_bar[s], dst, x, y);
+          for (int h = 0; h < kHalves; ++h) {
+            const int nh = n0 + h * kBN;  // this CTA's B rows of half h
+#pragma unroll
+            for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
+              void* dst = b_s + h * kBBytes + sl * kSlabBytes;
+              const int x = B_MN ? nh + sl * kMNe : k0, y = B_MN ? k0 : nh;
+              if (PAIR) tma_load_2d_pair(&tmB, fb, dst, x, y);
+              else tma_load_2d(&tmB, &full_bar[s], dst, x, y);
+            }
           }
           ++issued;
         }
@@ -320,8 +334,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t consumed = 0, local = 0;
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += units, ++local) {
-        const uint32_t buf = local & 1u;
-        const uint32_t aph = (local >> 1) & 1u;
+        const uint32_t buf = local % kAccBufs;
+        const uint32_t aph = (local / kAccBufs) & 1u;
         if (!wait_bar(&tempty_bar[buf], aph ^ 1u, ctl)) {
           ok = false;
           break;
@@ -344,16 +358,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t ad = A_MN ? sdesc_sw128(a_addr + j * (kUmmaK / 8) * 1024,
                                                    kSlabBytes, 1024)
                                      : sdesc_sw128(a_addr + j * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(b_addr + j * (kUmmaK / 8) * 1024,
-                                                   kSlabBytes, 1024)
-                                     : sdesc_sw128(b_addr + j * 32, 16, 1024);
             const uint32_t acc = (kb != ur.kb0 || j != 0) ? 1u : 0u;
-            if (PAIR) {
-              if (kEB == 2) umma_f16_pair(d_tmem, ad, bd, kIdesc, acc);
-              else umma_tf32_pair(d_tmem, ad, bd, kIdesc, acc);
-            } else {
-              if (kEB == 2) umma_f16(d_tmem, ad, bd, kIdesc, acc);
-              else umma_tf32(d_tmem, ad, bd, kIdesc, acc);
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+              const uint32_t bh = b_addr + h * kBBytes;
+              const uint64_t bd = B_MN ? sdesc_sw128(bh + j * (kUmmaK / 8) * 1024,
+                                                     kSlabBytes, 1024)
+                                       : sdesc_sw128(bh + j * 32, 16, 1024);
+              const uint32_t dh = d_tmem + h * kBN;
+              if (PAIR) {
+                if (kEB == 2) umma_f16_pair(dh, ad, bd, kIdesc, acc);
+                else umma_tf32_pair(dh, ad, bd, kIdesc, acc);
+              } else {
+                if (kEB == 2) umma_f16(dh, ad, bd, kIdesc, acc);
+                else umma_tf32(dh, ad, bd, kIdesc, acc);
+              }
             }
           }
           // frees the smem stage (in both CTAs of a pair) when these MMAs finish
@@ -442,8 +461,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const UnitRange ur = unit_range(t, p);
       int tm, tn;
       tile_coords(ur.tile, p, tm, tn);
-      const uint32_t buf = local & 1u;
-      const uint32_t aph = (local >> 1) & 1u;
+      const uint32_t buf = local % kAccBufs;
+      const uint32_t aph = (local / kAccBufs) & 1u;
       if (!wait_bar(&tfull_bar[buf], aph, ctl)) break;
       __syncwarp();
       tc_fence_after();
@@ -452,7 +471,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int grow = row0 + lane;
       const bool rv = grow < p.rows_valid;
       const bool warp_rows = row0 < p.rows_valid;  // any row of this warp's box exists
-      const int col0 = tn * kBN;
+      const int col0 = tn * kTileN;
 
       if (EPI == EPI_STATS) {
         const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
@@ -573,12 +592,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < kTileN / 32; ++c) {  // both halves: TMEM columns are contiguous
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (c == kBN / 32 - 1) release(buf);
+          if (c == kTileN / 32 - 1) release(buf);
           const int cb = col0 + c * 32;
           if (cb >= p.cols_valid) continue;
           if (EPI == EPI_STORE)
