@@ -261,3 +261,34 @@ def test_two_processes_over_gloo_on_one_gpu():
         assert r["row"] <= 1.0 and r["lse"] <= 1e-4, r
         assert r["dH"] <= GRAD_FRAC * r["dH_scale"], r
         assert r["dW"] <= GRAD_FRAC * r["dW_scale"], r
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_hidden_shards_with_every_option(dtype):
+    """Teacher-hidden shards with a per-token temperature, a mask, reverse-KL
+    mixing, several chunks and dW accumulation on top of existing values."""
+    w = _hidden(dtype=dtype, seed=40)
+    g = torch.Generator().manual_seed(40)
+    w.T = (0.6 + 2.0 * torch.rand(w.N, generator=g)).to(torch.float32).cuda()
+    kw = dict(_kw(w, chunk=64), reverse_weight=0.4)
+    Wt = kw.pop("Wt")
+    shards = [(0, 700), (700, 2048), (2048, 3001)]
+    base = torch.randn(w.W.shape, generator=g).cuda()
+    passes = [vp.ShardPass(w.H, w.W[a:b], v_begin=a, V_total=w.V, Wt=Wt[a:b],
+                           dW=base[a:b].clone(), accumulate_dW=True, want_row_loss=True,
+                           want_lse=True, **kw) for a, b in shards]
+    for k in range(len(passes[0].chunks)):
+        st = torch.cat([s.fwd_chunk(k) for s in passes])
+        sums = torch.cat([s.mid_chunk(k, st, 3, r) for r, s in enumerate(passes)])
+        for r, s in enumerate(passes):
+            s.bwd_chunk(k, st, 3, r, 0.9, sums)
+    ref = _oracle(w, reverse_weight=0.4, grad_loss=0.9)
+    loss = float(sum(s.loss for s in passes))
+    assert abs(loss - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"])
+    row = sum(s.row_loss for s in passes).cpu().numpy()
+    np.testing.assert_allclose(row, ref["row_loss"], rtol=5e-3, atol=2e-4)
+    dH32 = sum(s.dH32 for s in passes)
+    _check_grad(passes[0].cast_dH(dH32), ref["dH"], "dH")
+    dW = torch.cat([s.dW for s in passes]) - base
+    _check_grad(dW, ref["dW"], "dW")
+    assert all(ops.status(s.ws) == 0 for s in passes)
