@@ -54,8 +54,8 @@ def parse():
     ap.add_argument("--parallel", default="tokens", choices=["tokens", "vocab"],
                     help="tokens: each rank its own token shard, no collective (weak scaling); "
                          "vocab: the head split by vocabulary rows over the ranks, the same "
-                         "tokens on every rank, one statistics all-gather per chunk and an "
-                         "all-reduce of dH (strong scaling)")
+                         "tokens on every rank, one statistics all-gather per chunk (two with "
+                         "a reverse-KL weight) and an all-reduce of dH (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=0,
@@ -216,8 +216,8 @@ def gpu_arm(args):
         else:
             dist.init_process_group(backend, timeout=_pg_timeout())
     vocab = args.parallel == "vocab"
-    if vocab and (args.entry != "fused" or args.reverse_weight > 0):
-        raise SystemExit("--parallel vocab runs the fused pass with forward KL only")
+    if vocab and args.entry != "fused":
+        raise SystemExit("--parallel vocab runs the fused pass (kl_vp_* calls)")
     # vocabulary-parallel ranks share the tokens: the same seed everywhere
     w = make_workload(wl, args, dev, 0 if vocab else rank)
     args.N = w.N
