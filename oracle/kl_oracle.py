@@ -25,7 +25,7 @@ And the KDFlow abstract (thelatestinai.com/papers/2603.01875): full-vocabulary
 distillation with teacher logits recomputed from the teacher's final hidden
 states through a frozen copy of the teacher's output head.
 
-Readings where the pages are silent (all restated in the design doc):
+Readings where the pages are silent:
   R1 temperature T divides both student and teacher logits; no T^2 factor.
   R2 partial mass: q_i = exp(t_i/T - lse_t) with lse_t the teacher's full
      vocabulary log-sum-exp at the same T (supplied with the cache); the mass
