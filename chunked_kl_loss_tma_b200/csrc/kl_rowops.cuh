@@ -1,11 +1,11 @@
 // kl_rowops.cuh -- the SIMT (HBM-bound) steps of the fused KL loss.
 //
 // Source: "Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and
-// a Fused Chunked KL Loss", §3 "Offline distillation" (teacher-entropy, cross
-// and mass terms need only the cached support; log Z is the one full-vocabulary
-// reduction) and §3 "Offline implementations" (each chunk writes its scalar
-// log Z values and scatters over the K retained entries); KDFlow abstract for
-// the teacher-hidden mode.
+// a Fused Chunked KL Loss", §3 "Offline distillation" (apart from the student's
+// normaliser, every term of the top-K loss is a sum over the cached entries
+// alone) and §3 "Offline implementations" (the chunked variant keeps one
+// normaliser per token and adds its corrections at the cached positions only);
+// KDFlow abstract for the teacher-hidden mode.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>

@@ -9,8 +9,8 @@ once ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and a
 Fused Chunked KL Loss", §3 "Offline distillation" and App. A): teacher logits
 t = Ht . Wt^T of a separate random teacher head on separate random hidden
 states, its K largest entries (int32 index + fp32 logit, in descending order)
-and the teacher's full-vocabulary log-sum-exp of t/T, which lets the loss keep
-the cached entries' unnormalised partial mass.
+and the teacher's full-vocabulary log-sum-exp of t/T, with which the loss uses
+the cached entries' probabilities without renormalising them over the K.
 
 Workloads (sizes and distributions of the benchmark configurations):
   tiny          N=64, d=64, V=1000, fp32 H~N(0,1), W~N(0,0.05^2); K=8 cache from a

@@ -8,7 +8,7 @@
  * lse_s = log sum_j exp(s~_j), p_s = softmax(s~):
  *
  *   KL_TEACHER_TOPK, partial mass (teacher_lse != NULL; §3 "Offline
- *   distillation": the cached top-K keeps its unnormalised partial mass):
+ *   distillation": the cached probabilities are not renormalised over K):
  *       q_i = exp(t_i / T - lse_t),  m = sum_i q_i,
  *       l_n = sum_{i in S_n} q_i (log q_i - s~_{idx_i} + lse_s)
  *           = [sum q log q] - [sum q_i s~_{idx_i}] + m * lse_s

@@ -11,16 +11,18 @@ step):
 
 Source: "Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and a
 Fused Chunked KL Loss" (Ryskulov et al.), section-by-section summary page:
-  * §1 Introduction, "Fused, chunked KL loss": the objective is a forward KL
-    for knowledge distillation, over sparse top-K teacher distributions with
-    partially retained mass.
+  * §1 Introduction, "Fused, chunked KL loss": a forward-KL distillation
+    objective whose teacher side is a sparse top-K distribution that keeps
+    only part of the probability mass.
   * §3 Types of Knowledge Distillation, "Online distillation": dense teacher
     probabilities against student log-probabilities (forward KL(p_t || p_s)).
-  * §3 "Offline distillation": the cache holds the teacher's K largest
-    probabilities with their unnormalised partial mass retained; the student
-    side needs K gathered student log-probabilities and the scalar log Z.
-  * §3 "Offline implementations": the dense-reconstruction variant (scatter the
-    cached top-K into a dense teacher tensor) is the correctness baseline.
+  * §3 "Offline distillation": the cache stores the teacher's K most likely
+    tokens with probabilities that are not renormalised over those K; the
+    student contributes its log-probabilities at the K cached tokens and one
+    normaliser per token.
+  * §3 "Offline implementations": the reference variant expands the cache
+    into a dense teacher distribution over the vocabulary; the dense
+    reconstruction below is that check.
 And the KDFlow abstract (thelatestinai.com/papers/2603.01875): full-vocabulary
 distillation with teacher logits recomputed from the teacher's final hidden
 states through a frozen copy of the teacher's output head.
@@ -90,8 +92,7 @@ def logsumexp_rows(x):
     """log sum_j exp(x_j) per row, written as max + log sum exp(x - max).
 
     The shift by the row maximum is an exact identity, not an approximation.
-    This is the "scalar log Z over the vocabulary" of §3 "Offline
-    distillation"."""
+    This is the per-token student normaliser of §3 "Offline distillation"."""
     m = np.max(x, axis=1, keepdims=True)
     return (m + np.log(np.sum(np.exp(x - m), axis=1, keepdims=True)))[:, 0]
 
