@@ -11,9 +11,13 @@
 //   gemm STATS     S~ = H_c W^T / T  (tcgen05), split-V row statistics + gather
 //   row_reduce     lse_s, row loss
 //   dlogits_topk   S~ -> dS in place
-//   gemm STORE     dH_c = dS W
+//   gemm ACCUM     dH_c = dS W: wide 256 x 512 tiles, split-K fp32 parts
+//   splitk_reduce  the parts summed in a fixed order -> dH_c
 //   gemm ACCUM     dW (+)= dS^T H_c
-// then finalize_loss (masked mean).  No host synchronisation anywhere.
+// then finalize_loss (masked mean).  No host synchronisation anywhere.  The
+// teacher-hidden mode launches the STATS GEMM twice (student, teacher) and
+// dlogits_full instead of prep_topk / dlogits_topk; the vocabulary-parallel
+// calls (kl_vp_*) split the same sequence around per-chunk exchanges.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

@@ -8,12 +8,14 @@
 //                                     fp32 accumulation in TMEM)
 //
 //   EPI_STATS  logits tile S = H_c . W^T: per (row, 256-column tile) the
-//              online max and sum of 2^(s~ log2 e) and the cross term
+//              max and sum of 2^(s~ log2 e - max) and the cross term
 //              sum_i q_i s~_{idx_i} of the cached top-K entries that fall in
 //              the tile (gathered from the fp32 accumulator); optionally
-//              stores s~ = s / T to the chunk's logit buffer.
+//              stores s~ - max (the tile maximum, natural units) to the
+//              chunk's logit buffer.
 //   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
-//   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, add-reduced into dW across chunks.
+//   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, add-reduced into dW across chunks;
+//              also the fp32 split-K parts of dH.
 //   EPI_DLOGITS backward with the row lse already known (the split forward /
 //              backward path): dS = c (m exp(s~ - lse) - q [j in S]) formed from
 //              the fp32 accumulator and stored, with c = g / (n T) (0 on masked
@@ -34,7 +36,10 @@
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
 //   warp 5     TMEM allocator + MMA issuer (one thread).
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
-// i overlap the main loop of tile i + 1.
+// i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
+// the 512 columns with one 256 x 512 tile (see the template below).  In the
+// double-buffered variants waiting threads are parked by the hardware between
+// barrier polls rather than spinning.
 //
 // Every wait on an mbarrier is bounded (spin_limit clock cycles); when one
 // runs out the CTA records KL_ERR_TIMEOUT in *status, every role leaves its
