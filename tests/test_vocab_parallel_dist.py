@@ -1,5 +1,6 @@
 """Host logic of the vocabulary-parallel pass on CPU: shard boundaries, and
-`run_pass` driving two gloo ranks.
+`run_pass` driving two gloo ranks (top-K mode with one exchange per chunk, and
+teacher-hidden mode with a reverse-KL weight and two exchanges).
 
 Each rank's per-chunk compute here is a small numpy stand-in written from the
 decomposition the library uses (per-shard log-sum-exp and cross term, merged
@@ -178,3 +179,118 @@ def test_two_rank_vocabulary_parallel_pass_matches_whole_head_oracle():
         assert scale > 1e-3
         assert abs(dloss) < 1e-12 and drow < 1e-12 and dlse < 1e-12, rank
         assert ddH < 1e-12 and ddW < 1e-12, rank
+
+
+class NumpyHiddenShard:
+    """Stand-in for ShardPass in the teacher-hidden mode with a reverse-KL weight:
+    the two exchanges of run_pass (row lse's, then the sums A and U)."""
+
+    def __init__(self, H, W, Ht, Wt, v0, v1, T, mask, beta, chunk):
+        self.H, self.Ht, self.Ws, self.Wts = H, Ht, W[v0:v1], Wt[v0:v1]
+        self.T, self.mask, self.beta = T, mask, beta
+        self.n_valid = int(mask.sum())
+        N, d = H.shape
+        self.chunks = chunk_rows(N, chunk)
+        self.loss = torch.zeros((), dtype=torch.float64)
+        self.row_loss = torch.zeros(N, dtype=torch.float64)
+        self.lse_s = torch.zeros(N, dtype=torch.float64)
+        self.dH32 = torch.zeros(N, d, dtype=torch.float64)
+        self.dW = torch.zeros(v1 - v0, d, dtype=torch.float64)
+        self.two_exchanges = True
+        self.ws = None
+
+    def fwd_chunk(self, k):
+        c0, n = self.chunks[k]
+        rows = slice(c0, c0 + n)
+        self._s = self.H[rows] @ self.Ws.T / self.T
+        self._t = self.Ht[rows] @ self.Wts.T / self.T
+        return torch.tensor(np.stack([_lse(self._s, 1), _lse(self._t, 1)], 1))
+
+    def _merged(self, stats_all, P, n):
+        st = stats_all.numpy().reshape(P, n, 2)
+        return _lse(st[:, :, 0], 0), _lse(st[:, :, 1], 0)
+
+    def mid_chunk(self, k, stats_all, P, rank):
+        n = self.chunks[k][1]
+        ls, lt = self._merged(stats_all, P, n)
+        ps = np.exp(self._s - ls[:, None])
+        pt = np.exp(self._t - lt[:, None])
+        u = self._s - self._t
+        return torch.tensor(np.stack([np.sum(-pt * u, 1), np.sum(ps * u, 1)], 1))
+
+    def bwd_chunk(self, k, stats_all, P, rank, grad_loss=1.0, sums_all=None):
+        c0, n = self.chunks[k]
+        rows = slice(c0, c0 + n)
+        ls, lt = self._merged(stats_all, P, n)
+        sums = sums_all.numpy().reshape(P, n, 2)
+        A, U = sums[rank, :, 0], sums[rank, :, 1]
+        ubar = sums[:, :, 1].sum(0)
+        b = self.beta
+        keep = self.mask[rows] != 0
+        dl = (ls - lt) if rank == 0 else 0.0
+        self.lse_s[rows] = torch.tensor(ls)
+        self.row_loss[rows] = torch.tensor(np.where(keep, (1 - b) * (A + dl) + b * (U - dl), 0))
+        ps = np.exp(self._s - ls[:, None])
+        pt = np.exp(self._t - lt[:, None])
+        u = self._s - self._t
+        coef = np.where(keep, grad_loss / self.n_valid / self.T, 0.0)
+        dS = coef[:, None] * ((1 - b) * (ps - pt) + b * ps * (u - ubar[:, None]))
+        self.dH32[rows] = torch.tensor(dS @ self.Ws)
+        self.dW += torch.tensor(dS.T @ self.H[rows])
+        if c0 + n == self.H.shape[0]:
+            self.loss.fill_(float(self.row_loss.sum()) / self.n_valid)
+
+    def dH_rows(self, k):
+        c0, n = self.chunks[k]
+        return self.dH32[c0:c0 + n]
+
+    def cast_dH(self):
+        return self.dH32.clone()
+
+    def empty_pass(self):
+        self.dW.zero_()
+
+
+def _hidden_worker(rank, world, port, q):
+    import oracle
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(11)  # the same whole problem on every rank
+        N, d, d_t, V, T, beta = 19, 5, 7, 29, 1.7, 0.4
+        H, Ht = rng.normal(size=(N, d)), rng.normal(size=(N, d_t))
+        W, Wt = rng.normal(scale=0.5, size=(V, d)), rng.normal(scale=0.5, size=(V, d_t))
+        mask = (rng.random(N) > 0.2).astype(np.uint8)
+        v0, v1 = vocab_shard(V, world, rank, align=8)
+        shard = NumpyHiddenShard(H, W, Ht, Wt, v0, v1, T, mask, beta, chunk=6)
+        out = run_pass(shard, TorchComm(), grad_loss=1.3)
+        ref = oracle.kl_loss(H, W, T=T, mask=mask, mode="hidden", Ht=Ht, Wt=Wt,
+                             reverse_weight=beta, grad_loss=1.3)
+        q.put((rank, float(out["loss"]) - ref["loss"],
+               float(np.max(np.abs(out["row_loss"].numpy() - ref["row_loss"]))),
+               float(np.max(np.abs(out["dH"].numpy() - ref["dH"]))),
+               float(np.max(np.abs(out["dW"].numpy() - ref["dW"][v0:v1]))),
+               float(np.max(np.abs(ref["dH"])))))
+    except Exception as e:  # report instead of leaving the parent waiting
+        q.put((rank, repr(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_reverse_kl_pass_with_two_exchanges_matches_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_hidden_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in res:
+        assert len(r) == 6, r
+        rank, dloss, drow, ddH, ddW, scale = r
+        assert scale > 1e-3
+        assert abs(dloss) < 1e-12 and drow < 1e-12 and ddH < 1e-12 and ddW < 1e-12, r
