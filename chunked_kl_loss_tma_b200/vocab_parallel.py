@@ -80,7 +80,8 @@ class ShardPass:
         if n < 0:
             raise ValueError("invalid vocabulary-parallel problem")
         self.chunks = chunk_rows(H.shape[0], kw.get("chunk_tokens", 0))
-        assert len(self.chunks) == n, (len(self.chunks), n)
+        if len(self.chunks) != n:  # the library's chunking and this module's must agree
+            raise RuntimeError(f"chunk count mismatch: {len(self.chunks)} here, {n} in the library")
         N, d = H.shape
         self.loss = torch.zeros((), dtype=torch.float32, device=dev)
         self.row_loss = torch.empty(N, dtype=torch.float32, device=dev) if want_row_loss else None
