@@ -1,7 +1,6 @@
 """C-ABI checks that need no GPU: the library loads, exports every function the
 header declares, sizes workspaces as O(chunk * V + N), and rejects bad
 arguments on the host before touching a device."""
-import ctypes
 import os
 import re
 

@@ -9,7 +9,6 @@ is at least -log of the student's mass on the support, the result does not
 depend on how many rows the oracle evaluates per block, and the gradient of H
 matches central finite differences."""
 import numpy as np
-import pytest
 import scipy.special
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st

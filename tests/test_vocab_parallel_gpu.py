@@ -10,7 +10,6 @@ import pytest
 import torch
 
 import oracle
-from chunked_kl_loss_tma_b200 import _lib as L
 from chunked_kl_loss_tma_b200 import ops
 from chunked_kl_loss_tma_b200 import vocab_parallel as vp
 from chunked_kl_loss_tma_b200 import workloads as wl

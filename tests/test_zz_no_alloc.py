@@ -10,7 +10,6 @@ the tolerances the parity tests use; it also checks the size and dtype limits.
 
 The file name makes pytest collect it last, so a failure here does not stop a
 `-x` run before the other tests."""
-import ctypes
 
 import numpy as np
 import pytest
