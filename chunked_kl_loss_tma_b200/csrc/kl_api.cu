@@ -204,6 +204,13 @@ struct Plan {
   // current chunk of H or Ht) and K-major copies W^T [d][Vp], dS^T [V][Cp],
   // H_c^T [d][Cp] for the gradient contractions.
   int64_t Cp = 0;
+  // bf16 top-K: the logits pass stores exponentials and the gradient
+  // contractions form dS from them as their operand stages arrive (no dlogits
+  // pass); fp32 keeps the dlogits pass (its operands are transposed copies)
+  bool xf = false;
+  int64_t Cx = 0;          // (xf) row stride of the transposed dS scales: C rounded up to 64
+  size_t off_xsc = 0;      // (xf) dS scales [tiles_v][Cx] fp32
+  size_t off_ubar = 0;     // (hidden) u_bar per chunk row
   int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
   size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
   size_t off_wr = 0, off_wtr = 0, off_xr = 0, off_wT = 0, off_sT = 0, off_hT = 0;
@@ -297,8 +304,12 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (pl.C < 1) pl.C = 1;
   pl.Vp = cdiv(p->V, 8) * 8;
   pl.tiles_v = static_cast<int>(cdiv(p->V, kBN));
-  const bool need_sbuf = entry != KL_ENTRY_FWD || pl.hidden;
-  const bool need_stats = entry != KL_ENTRY_BWD;
+  pl.xf = pl.eb == 2 && !pl.hidden;
+  // student logits / dS chunk: wherever dS is formed (not the forward alone)
+  const bool need_sbuf = entry != KL_ENTRY_FWD;
+  // tile statistics: every pass that computes them (the top-K backward forms
+  // dS in its recompute epilogue from the known lse and needs none)
+  const bool need_stats = entry != KL_ENTRY_BWD || pl.hidden;
   size_t off = 256;  // Scalars
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -307,10 +318,16 @@ Plan make_plan(const kl_problem* p, int entry) {
   };
   const size_t buf = static_cast<size_t>(pl.C) * pl.Vp * pl.eb;
   if (need_sbuf) pl.off_sbuf = take(buf);
-  if (need_sbuf && pl.hidden) pl.off_tbuf = take(buf);
+  // teacher logits chunk, fp32: the student pass forms the loss sums from it
+  if (pl.hidden) pl.off_tbuf = take(static_cast<size_t>(pl.C) * pl.Vp * 4);
   if (need_stats) pl.off_ps = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
   if (need_stats && pl.hidden)
     pl.off_pt = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
+  if (pl.hidden && entry != KL_ENTRY_FWD) pl.off_ubar = take(static_cast<size_t>(pl.C) * 4);
+  if (pl.xf && entry == KL_ENTRY_FWD_BWD) {
+    pl.Cx = cdiv(pl.C, 64) * 64;
+    pl.off_xsc = take(static_cast<size_t>(pl.tiles_v) * pl.Cx * 4);
+  }
   if (!pl.hidden) {
     pl.off_sidx = take(static_cast<size_t>(pl.C) * p->K * 4);
     pl.off_sq = take(static_cast<size_t>(pl.C) * p->K * 4);
@@ -346,10 +363,10 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE>;
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -365,7 +382,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(XF ? kGemmThreadsXf : kGemmThreads);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = st;
   if (PAIR) {
@@ -422,10 +439,16 @@ int prepare_heads(Ctx& c) {
   return KL_OK;
 }
 
+// Logits pass over one chunk: S~ = X_c . Wh^T / T with the tile statistics in
+// `partials`.  store: STORE_NONE, STORE_SHIFTED (s~ - tile max into `out`, fp32
+// when out_f32, else the input type) or STORE_EXP (bf16 exponentials).  tbuf /
+// tpart: the teacher pass's stored tile and statistics (student pass of the
+// teacher-hidden mode: the tile sums A and U go to partials .z / .w).
 template <typename Elem>
 int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, int64_t Cn,
-                void* out, float4* partials, const int* sidx, const float* sq, int ktop,
-                const char* name) {
+                void* out, int store, bool out_f32, float4* partials, const int* sidx,
+                const float* sq, int ktop, const char* name, const float* tbuf = nullptr,
+                const float4* tpart = nullptr) {
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   CUtensorMap ma, mb;
@@ -439,8 +462,11 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
       !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2))
     return KL_ERR_CUDA;
-  if (out != nullptr) {
-    if (!make_out_map(&mc, out, p->dtype, p->V, Cn, c.pl.Vp * sizeof(Elem))) return KL_ERR_CUDA;
+  if (store != STORE_NONE) {
+    const bool f32 = out_f32 && store == STORE_SHIFTED;
+    if (!make_out_map(&mc, out, f32 ? KL_DTYPE_F32 : p->dtype, p->V, Cn,
+                      c.pl.Vp * (f32 ? 4 : sizeof(Elem))))
+      return KL_ERR_CUDA;
   } else {
     mc = mb;  // statistics only: the output map is not used
   }
@@ -449,7 +475,8 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.tiles_n = c.pl.tiles_v;
   gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
   gp.m_fastest = 1;
-  gp.store = out != nullptr;
+  gp.store = store;
+  gp.out_f32 = out_f32 ? 1 : 0;
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
   gp.scale = c.invT;
@@ -458,6 +485,9 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.sidx = sidx;
   gp.sq = sq;
   gp.ktop = ktop;
+  gp.tbuf = tbuf;
+  gp.tld = c.pl.Vp;
+  gp.tpart = tpart;
   gp.status = &c.sc->status;
   gp.spin_limit = spin_limit();
   return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, mc, gp,
@@ -568,17 +598,25 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
                                                  2.0 * Cn * p->V * dx);
 }
 
-// dH_f32: write dH as fp32 (a vocabulary shard's partial sum) whatever Elem is.
-template <typename Elem>
-int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
-               bool dH_f32 = false) {
-  if (sizeof(Elem) == 4)
-    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
+// dH_c = dS . W and dW (+)= dS^T . H_c for chunk rows [c0, c0 + Cn) from the
+// chunk buffer dS.  dH_f32: write dH as fp32 (a vocabulary shard's partial sum)
+// whatever Elem is.  XF = 1: the buffer holds the logits pass's exponentials,
+// patched at the cached columns (xf_patch_kernel), and the two contractions
+// form dS = scale * e in shared memory with the per-(tile, row) scales xf_sc.
+template <typename Elem, int XF>
+int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+                    bool dH_f32, const float* xf_sc) {
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   constexpr int kMNe = kRowBytes / sizeof(Elem);
   const int64_t d = p->d;
   const uint64_t ldS = c.pl.Vp * sizeof(Elem);
+  auto set_xf = [&](GemmParams& gp) {
+    if (!XF) return;
+    gp.xf_sc = xf_sc;
+    gp.xf_ld = c.pl.Cx;
+    gp.xf_rows = static_cast<int>(Cn);
+  };
   // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.  When the
   // output has too few tiles to fill the GPU, V is split into ksplit parts whose
   // fp32 partial products are summed in a fixed order afterwards.
@@ -596,6 +634,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
+    set_xf(gp);
     int ks = choose_ksplit(static_cast<int64_t>(gp.tiles_m) * gp.tiles_n, gp.num_kb, c.sms / 2);
     if (ks > c.pl.ksplit_dh) ks = c.pl.ksplit_dh;
     if (ks > 1) {
@@ -610,8 +649,8 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
-                                                    2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d)));
       LaunchScope ls("splitk_reduce", c.st, 0,
                      (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
       if (dH_f32)
@@ -627,15 +666,15 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
-                                                    2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
                         d * sizeof(Elem)))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc, gp,
-                                                    2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d)));
     }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
@@ -656,10 +695,24 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
-                                                  2.0 * Cn * p->V * d)));
+    set_xf(gp);
+    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1, 0, XF>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
+                                                         2.0 * Cn * p->V * d)));
   }
   return KL_OK;
+}
+
+// dH_f32: write dH as fp32 (a vocabulary shard's partial sum) whatever Elem is.
+// xf_sc != nullptr: dS is formed in the contractions' operand path (bf16).
+template <typename Elem>
+int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+               bool dH_f32 = false, const float* xf_sc = nullptr) {
+  if (sizeof(Elem) == 4)
+    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
+  using B = __nv_bfloat16;
+  B* b = reinterpret_cast<B*>(dS);
+  return xf_sc != nullptr ? gemm_grads_bf16<B, 1>(c, b, c0, Cn, dH, dW, beta, dH_f32, xf_sc)
+                          : gemm_grads_bf16<B, 0>(c, b, c0, Cn, dH, dW, beta, dH_f32, nullptr);
 }
 
 int launch_count_valid(Ctx& c) {
@@ -746,24 +799,87 @@ int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* ls
   return KL_LAUNCHED();
 }
 
+// dS in place over the student buffer, teacher-hidden mode (one CTA per row).
 template <typename Elem>
-int launch_dlogits_full(Ctx& c, Elem* S, const Elem* Tt, int64_t c0, int64_t Cn,
-                        const float* lse_s, const float* lse_t, const float* g_dev, float g_host,
-                        float* row_loss, int write_grad, const float4* part_s,
-                        const float4* part_t, int add_lse = 1, int phase = kDlfBoth,
-                        float* sums_out = nullptr, const float* sums_all = nullptr, int P = 1,
-                        int rank = 0) {
+int launch_dlogits_full(Ctx& c, Elem* S, const float* Tt, int64_t c0, int64_t Cn,
+                        const float* lse_s, const float* lse_t, const float* ubar,
+                        const float* g_dev, float g_host) {
   const kl_problem* p = c.p;
-  LaunchScope ls("dlogits_full", c.st, 0,
-                 ((write_grad ? 3.0 : 2.0) + (p->reverse_weight > 0.f && write_grad ? 2.0 : 0.0)) *
-                     Cn * p->V * sizeof(Elem));
+  LaunchScope ls("dlogits_full", c.st, 0, (2.0 * sizeof(Elem) + 4.0) * Cn * p->V);
   dlogits_full_kernel<Elem><<<static_cast<unsigned>(Cn), kDlogitsFullThreads, 0, c.st>>>(
-      S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0,
+      S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0, ubar,
       p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
-      p->T_row ? p->T_row + c0 : nullptr, row_loss ? row_loss + c0 : nullptr, write_grad,
-      p->reverse_weight, part_s, part_t, c.pl.tiles_v, add_lse, phase, sums_out, sums_all, P,
-      rank, static_cast<int>(Cn));
+      p->T_row ? p->T_row + c0 : nullptr, p->reverse_weight,
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_ps),
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_pt), c.pl.tiles_v);
   return KL_LAUNCHED();
+}
+
+// dS from the stored exponentials of chunk rows [c0, c0 + Cn) (top-K, bf16):
+// the cached columns' corrections folded into the buffer S, then the
+// transposed per-(tile, row) scales.  lse: the whole problem's rows.  Returns
+// the scales for gemm_grads.
+int launch_xf_prep(Ctx& c, __nv_bfloat16* S, int64_t c0, int64_t Cn, const float* lse,
+                   const float* g_dev, float g_host, const float** xf_sc) {
+  const kl_problem* p = c.p;
+  const float4* part = reinterpret_cast<const float4*>(c.ws + c.pl.off_ps);
+  const float2* rinfo = reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo);
+  const uint8_t* mask = p->mask ? p->mask + c0 : nullptr;
+  const float* T_row = p->T_row ? p->T_row + c0 : nullptr;
+  float* sc_out = reinterpret_cast<float*>(c.ws + c.pl.off_xsc);
+  {
+    LaunchScope ls("xf_patch", c.st, 0, static_cast<double>(Cn) * p->K * 16);
+    xf_patch_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
+        S, c.pl.Vp, part, c.pl.tiles_v, static_cast<int>(Cn), static_cast<int>(p->V), lse + c0,
+        mask, rinfo, reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+        reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT,
+        T_row);
+    KL_TRY(KL_LAUNCHED());
+  }
+  LaunchScope ls("xf_scales", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 20);
+  xf_scales_kernel<<<static_cast<unsigned>(cdiv(Cn, 32)), 256, 0, c.st>>>(
+      part, c.pl.tiles_v, static_cast<int>(Cn), lse + c0, mask, rinfo, c.sc, g_dev, g_host,
+      c.invT, T_row, sc_out, c.pl.Cx);
+  *xf_sc = sc_out;
+  return KL_LAUNCHED();
+}
+
+// Teacher-hidden row sums of chunk rows [c0, c0 + Cn) (hidden_sums_kernel).
+// lse_*_in: given log-sum-exps (whole arrays, or nullptr to merge them from the
+// tile statistics into lse_*_out); the other outputs as the kernel's, each
+// optional; sums_out / sums_all are per chunk ([rows] / [P][rows] pairs).
+int launch_hidden_sums(Ctx& c, int64_t c0, int64_t Cn, const float* lse_s_in,
+                       const float* lse_t_in, float* lse_s_out, float* lse_t_out, int add_lse,
+                       float* row_loss, float* sums_out, float* ubar_out,
+                       const float* sums_all = nullptr, int P = 1) {
+  const kl_problem* p = c.p;
+  LaunchScope ls("hidden_sums", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 32);
+  hidden_sums_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_ps),
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_pt), c.pl.tiles_v, static_cast<int>(Cn),
+      lse_s_in ? lse_s_in + c0 : nullptr, lse_t_in ? lse_t_in + c0 : nullptr,
+      lse_s_out ? lse_s_out + c0 : nullptr, lse_t_out ? lse_t_out + c0 : nullptr,
+      p->mask ? p->mask + c0 : nullptr, p->reverse_weight, add_lse,
+      row_loss ? row_loss + c0 : nullptr, sums_out, ubar_out, sums_all, P);
+  return KL_LAUNCHED();
+}
+
+// Teacher-hidden logits of one chunk: the teacher pass (fp32 t~ - tile max into
+// the teacher buffer, statistics), then the student pass (statistics and the
+// tile sums A, U formed against the teacher tile; s~ - tile max stored into
+// the student buffer when store_student).
+template <typename Elem>
+int hidden_logits(Ctx& c, int64_t c0, int64_t Cn, bool store_student) {
+  const kl_problem* p = c.p;
+  float* Tt = reinterpret_cast<float*>(c.ws + c.pl.off_tbuf);
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, STORE_SHIFTED, true, pt,
+                           nullptr, nullptr, 0, "gemm_teacher_logits"));
+  return gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn,
+                           store_student ? c.ws + c.pl.off_sbuf : nullptr,
+                           store_student ? STORE_SHIFTED : STORE_NONE, sizeof(Elem) == 4, ps,
+                           nullptr, nullptr, 0, "gemm_logits_stats", Tt, pt);
 }
 
 int launch_finalize(Ctx& c, const float* row_loss, float* loss) {
@@ -810,23 +926,15 @@ int run_fwd(Ctx& c, float* loss, float* lse_s, float* lse_t, float* row_loss) {
     const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
     if (!c.pl.hidden) {
       KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, nullptr, ps,
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, nullptr, STORE_NONE, false, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                                "gemm_logits_stats"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
     } else {
-      Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
-      Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
-      float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
-                               "gemm_logits_stats"));
-      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
-                               "gemm_teacher_logits"));
-      KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
-      KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, 0.f, rl, 0, ps,
-                                       pt));
+      KL_TRY(hidden_logits<Elem>(c, c0, Cn, false));
+      KL_TRY(launch_hidden_sums(c, c0, Cn, nullptr, nullptr, lse_s, lse_t, 1, rl, nullptr,
+                                nullptr));
     }
   }
   return launch_finalize(c, rl, loss);
@@ -839,7 +947,6 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
   KL_TRY(launch_count_valid(c));  // also resets the status word
   if (p->N == 0) return accumulate ? KL_OK : launch_fill(c, dW, p->V * p->d, 0.f);
   Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
-  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
   KL_TRY(prepare_heads(c));
   if (sizeof(Elem) == 4)
     KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
@@ -850,13 +957,13 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
       KL_TRY(launch_prep(c, c0, Cn));
       KL_TRY(gemm_dlogits<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
     } else {
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, nullptr, nullptr, nullptr, 0,
-                               "gemm_logits_recompute"));
-      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, nullptr, nullptr, nullptr,
-                               0, "gemm_teacher_logits"));
-      // backward: logits were recomputed without tile statistics (not shifted)
-      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, g_dev, g_host, nullptr,
-                                       1, nullptr, nullptr));
+      // both logits recomputed; u_bar from the given lse's
+      float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
+      KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
+      KL_TRY(launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, 1, nullptr, nullptr,
+                                ubar));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                       c0, Cn, lse_s, lse_t, ubar, g_dev, g_host));
     }
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
   }
@@ -871,9 +978,7 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
   float* lse_s = reinterpret_cast<float*>(c.ws + c.pl.off_lse_s);
   float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
   Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
-  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
-  float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
   KL_TRY(launch_count_valid(c));
   if (p->N == 0) {
     if (!accumulate) KL_TRY(launch_fill(c, dW, p->V * p->d, 0.f));
@@ -885,24 +990,31 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
                             reinterpret_cast<float*>(c.ws + c.pl.off_wT), c.pl.Vp, p->V, p->d));
   for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
     const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
+    const int beta = (accumulate || c0 > 0) ? 1 : 0;
     if (!c.pl.hidden) {
       KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps,
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S,
+                               c.pl.xf ? STORE_EXP : STORE_SHIFTED, sizeof(Elem) == 4, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                                "gemm_logits_stats"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
+      if (c.pl.xf) {
+        const float* xsc = nullptr;
+        KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
+                              &xsc));
+        KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, false, xsc));
+        continue;
+      }
       KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
     } else {
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
-                               "gemm_logits_stats"));
-      KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
-                               "gemm_teacher_logits"));
-      KL_TRY(launch_row_reduce(c, ps, c0, Cn, false, lse_s, nullptr));
-      KL_TRY(launch_row_reduce(c, pt, c0, Cn, false, lse_t, nullptr));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1, ps, pt));
+      float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
+      KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
+      KL_TRY(launch_hidden_sums(c, c0, Cn, nullptr, nullptr, lse_s, lse_t, 1, rl, nullptr, ubar));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                       c0, Cn, lse_s, lse_t, ubar, nullptr, g));
     }
-    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta));
   }
   return launch_finalize(c, rl, loss);
 }
@@ -933,18 +1045,15 @@ int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
   if (!c.pl.hidden) {
     KL_TRY(launch_prep(c, c0, Cn));
-    KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps,
+    KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S,
+                             c.pl.xf ? STORE_EXP : STORE_SHIFTED, sizeof(Elem) == 4, ps,
                              reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                              reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                              "gemm_logits_stats"));
     return launch_row_stats(c, ps, Cn, stats, 0, true);
   }
-  Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
   float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
-  KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, ps, nullptr, nullptr, 0,
-                           "gemm_logits_stats"));
-  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, pt, nullptr, nullptr, 0,
-                           "gemm_teacher_logits"));
+  KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
   KL_TRY(launch_row_stats(c, ps, Cn, stats, 0, false));
   return launch_row_stats(c, pt, Cn, stats, 1, false);
 }
@@ -966,7 +1075,8 @@ int launch_vp_merge(Ctx& c, int64_t c0, int64_t Cn, const float* stats_all, int 
 }
 
 // Teacher-hidden mode with a reverse-KL weight: this shard's sums (A, U) of
-// chunk k, written to sums_out [rows][2].
+// chunk k over its columns, from the tile statistics and the whole-vocabulary
+// lse's, written to sums_out [rows][2].
 template <typename Elem>
 int run_vp_mid_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank,
                      float* sums_out) {
@@ -974,12 +1084,10 @@ int run_vp_mid_chunk(Ctx& c, int64_t k, const float* stats_all, int P, int rank,
   chunk_rows(c, k, &c0, &Cn);
   float* rl = reinterpret_cast<float*>(c.ws + c.pl.off_rl);
   KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, nullptr, rl));
-  return launch_dlogits_full<Elem>(
-      c, reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf), reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf),
-      c0, Cn, reinterpret_cast<float*>(c.ws + c.pl.off_lse_s),
-      reinterpret_cast<float*>(c.ws + c.pl.off_lse_t), nullptr, 0.f, nullptr, 0,
-      reinterpret_cast<float4*>(c.ws + c.pl.off_ps), reinterpret_cast<float4*>(c.ws + c.pl.off_pt),
-      0, kDlfSums, sums_out, nullptr, P, rank);
+  const float* lse_s = reinterpret_cast<const float*>(c.ws + c.pl.off_lse_s);
+  const float* lse_t = reinterpret_cast<const float*>(c.ws + c.pl.off_lse_t);
+  return launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, 0, nullptr, sums_out,
+                            nullptr);
 }
 
 template <typename Elem>
@@ -994,18 +1102,29 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sum
   float* lse_t = c.pl.hidden ? reinterpret_cast<float*>(c.ws + c.pl.off_lse_t) : nullptr;
   Elem* S = reinterpret_cast<Elem*>(c.ws + c.pl.off_sbuf);
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  const int beta = (accumulate || k > 0) ? 1 : 0;
   KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, lse_user, rl));
   if (!c.pl.hidden) {
-    KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
+    if (c.pl.xf) {
+      const float* xsc = nullptr;
+      KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
+                            &xsc));
+      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true, xsc));
+    } else {
+      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
+      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
+    }
   } else {
-    Elem* Tt = reinterpret_cast<Elem*>(c.ws + c.pl.off_tbuf);
-    float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
-    const bool split = p->reverse_weight > 0.f;  // u_bar came through the second exchange
-    KL_TRY(launch_dlogits_full<Elem>(c, S, Tt, c0, Cn, lse_s, lse_t, nullptr, g, rl, 1, ps, pt,
-                                     rank == 0 ? 1 : 0, split ? kDlfGrad : kDlfBoth, nullptr,
-                                     sums_all, P, rank));
+    // this shard's A, U (its row-loss share) and u_bar, the sum of every shard's
+    // U when the reverse KL needs it (its sums came through the second exchange)
+    float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
+    const bool mixed = p->reverse_weight > 0.f;
+    KL_TRY(launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, rank == 0 ? 1 : 0, rl,
+                              nullptr, ubar, mixed ? sums_all : nullptr, P));
+    KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                     c0, Cn, lse_s, lse_t, ubar, nullptr, g));
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
   }
-  KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || k > 0) ? 1 : 0, true));
   if (c0 + Cn == p->N) KL_TRY(launch_finalize(c, rl, loss));
   return KL_OK;
 }
@@ -1210,22 +1329,14 @@ int kl_profile_end(kl_profile_entry* out, int max_entries) {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[KL_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-uint8_t* g_noalloc_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.
+// Device address of the scratch array for the current device and context.  It
+// is looked up on every call (a cheap runtime query) rather than cached, so a
+// context that was destroyed and created again never gets a stale address.
 int noalloc_scratch(uint8_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KL_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-      return KL_ERR_CUDA;
-    g_noalloc_ptr[dev] = static_cast<uint8_t*>(ptr);
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+    return KL_ERR_CUDA;
+  *out = static_cast<uint8_t*>(ptr);
   return KL_OK;
 }
 }  // namespace

@@ -1,8 +1,9 @@
 // kl_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for the three
 // contractions of the fused KL loss, with the loss arithmetic fused into the
-// epilogue ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits
-// and a Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection
-// is integrated into the loss and each logit chunk is transient).
+// epilogue and, for the gradient contractions, into the operand path
+// ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and a
+// Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection is
+// integrated into the loss and each logit chunk is transient).
 //
 //   C[M, N] = A[M, K] . B[N, K]^T   (bf16 -> kind::f16, fp32 -> kind::tf32;
 //                                     fp32 accumulation in TMEM)
@@ -10,9 +11,13 @@
 //   EPI_STATS  logits tile S = H_c . W^T: per (row, 256-column tile) the
 //              max and sum of 2^(s~ log2 e - max) and the cross term
 //              sum_i q_i s~_{idx_i} of the cached top-K entries that fall in
-//              the tile (gathered from the fp32 accumulator); optionally
-//              stores s~ - max (the tile maximum, natural units) to the
-//              chunk's logit buffer.
+//              the tile (gathered from the fp32 accumulator).  Optionally
+//              stores s~ - max (store = 1; natural units) or the exponentials
+//              2^(s~ log2 e - max) themselves (store = 2), which the gradient
+//              contractions scale into dS as their operand stages arrive.  In
+//              the teacher-hidden mode the student pass also reads the
+//              teacher tile (stored fp32 by the teacher pass) and forms the
+//              tile's sums sum p_t (t~ - s~) and sum p_s (s~ - t~) from fp32.
 //   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
 //   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, add-reduced into dW across chunks;
 //              also the fp32 split-K parts of dH.
@@ -25,16 +30,20 @@
 // tcgen05.mma.cta_group::1; PAIR = 1, a cluster of two CTAs (one per SM)
 // computes a 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA loads its
 // own 128 rows of A and its own 128-row half of B, only the leader CTA issues
-// the MMAs, both CTAs' loads complete on the leader's barriers, the leader's
-// commits arrive on both CTAs' barriers, and each CTA's epilogue reads its own
-// 128 accumulator rows from its own TMEM.  The pair halves the operand bytes
-// each SM stages per MMA.
+// the MMAs, the leader's commits arrive on both CTAs' barriers, and each CTA's
+// epilogue reads its own 128 accumulator rows from its own TMEM.  The pair
+// halves the operand bytes each SM stages per MMA.
 //
 // Roles (192 threads, one CTA per SM, grid-strided over output tiles):
 //   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
-//   warp 5     TMEM allocator + MMA issuer (one thread).
+//   warp 5     TMEM allocator + MMA issuer (one thread);
+//   warps 6-9  (XF = 1 only) operand transform: turn the A stage -- the
+//              stored exponentials e = 2^(s~ log2 e - tile max) of a logit
+//              chunk -- into dS = scale(row, tile) * e - c q at the cached
+//              entries, in shared memory, before the MMAs read it.  This is
+//              the dlogits step of the loss without its own pass over HBM.
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
 // the 512 columns with one 256 x 512 tile (see the template below).  In the
@@ -42,9 +51,11 @@
 // barrier polls rather than spinning.
 //
 // Every wait on an mbarrier is bounded (spin_limit clock cycles); when one
-// runs out the CTA records KL_ERR_TIMEOUT in *status, every role leaves its
-// loop, in-flight copies and MMAs are drained (again with a bound) and TMEM is
-// released before the CTA exits.
+// runs out the CTA records KL_ERR_TIMEOUT in *status and raises the abort flag
+// of both CTAs of its pair, every role leaves its loop, the MMAs already
+// issued are drained, and after both CTAs of the pair have stopped, the copies
+// already issued are drained (again with a bound) before TMEM is released and
+// the CTAs exit.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -61,9 +72,10 @@ constexpr int kATileBytes = kBM * kRowBytes;
 constexpr int kBTileBytes = kBN * kRowBytes;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
+constexpr int kGemmThreadsXf = 320;  // + four operand-transform warps
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kRingBytes = kStages * kStageBytes;          // 192 KB operand ring
-constexpr int kBarrierRegion = 1024;                        // barriers, TMEM slot, flags
+constexpr int kBarrierRegion = 2048;                        // barriers, TMEM slot, flags, slots
 constexpr int kStageOutBytes = 4096;                        // one 32 x 32 fp32 output box
 constexpr int kStagingBytes = 4 * 2 * kStageOutBytes;       // 4 epilogue warps x 2 buffers
 constexpr int kGemmSmemBytes = 1024 /*align*/ + kRingBytes + kBarrierRegion + kStagingBytes;
@@ -77,22 +89,37 @@ constexpr int kStatusTimeout = 8;  // KL_ERR_TIMEOUT
 // finish on their own, and the CTA must not leave before they do.
 constexpr long long kDrainLimit = 1LL << 31;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2f = 0.6931471805599453f;
 
 enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3 };
+// EPI_STATS store modes
+enum { STORE_NONE = 0, STORE_SHIFTED = 1, STORE_EXP = 2 };
 
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
-  int store;           // STATS: store s~ through the output map (0 = statistics only)
+  int store;           // STATS: STORE_NONE / STORE_SHIFTED / STORE_EXP
+  int out_f32;         // STATS, STORE_SHIFTED: the output map holds fp32
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
   float scale;         // STATS / DLOGITS: 1 / T
   const float* T_row;  // STATS / DLOGITS: per-row temperature (chunk rows), or nullptr
   int beta;            // ACCUM: 0 overwrite, 1 accumulate
-  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross, 0)
-  const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
-  const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
+  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross | A, gather start | U)
+  const int* sidx;     // STATS gather / XF corrections: [rows][ktop] ascending ids,
+                       // INT_MAX = empty
+  const float* sq;     // STATS gather / XF corrections: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
+  // STATS, student pass of the teacher-hidden mode: the teacher tile stored by
+  // the teacher pass (t~ - tile max, fp32, row stride tld) and its statistics
+  const float* tbuf;
+  int64_t tld;
+  const float4* tpart;
+  // XF: scale of dS per (256-column tile, logit row), [tiles][xf_ld] fp32
+  // (xf_ld a multiple of 64), so that dS = scale * e for the stored e
+  const float* xf_sc;
+  int64_t xf_ld;
+  int xf_rows;         // logit rows (tokens) that exist
   // DLOGITS: per-row lse (natural units), (m, .) per row, mask, and the scalars
   // of c = g / (n T): the loss normaliser n, and g (device pointer or value)
   const float* lse;
@@ -127,11 +154,12 @@ struct Ctl {
   int* status;
   long long limit;
   volatile int* abort_flag;
+  uint32_t peer_abort;  // shared::cluster address of the other CTA's flag (0: none)
 };
 
 // Bounded wait for the phase of the given parity; false when the CTA aborted.
 // park: let the hardware park the waiting thread between polls.
-constexpr uint32_t kParkNs = 1000000;
+constexpr uint32_t kParkNs = 100;
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c,
                                          bool park = false) {
   auto poll = [&]() {
@@ -143,6 +171,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
     if (*c.abort_flag) return false;
     if (clock64() - t0 > c.limit) {
       *c.abort_flag = 1;
+      if (c.peer_abort != 0u) st_cluster_u32(c.peer_abort, 1u);  // stop the pair together
       atomicCAS(c.status, 0, kStatusTimeout);
       return false;
     }
@@ -202,18 +231,48 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// XF: one 128-byte row of a dS operand stage (64 bf16 values of one logit row
+// within one 256-column tile), x -> x * scale in place with packed bf16x2
+// multiplies (scale rounded to bf16: with the product's rounding, 2^-8
+// relative error per entry).  The chunks are visited in the row's swizzled
+// order (chunk j at position j ^ sw) so that the 32 rows a warp's lanes touch
+// at once hit all 32 banks.
+__device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 scale2) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint4* cp = reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4));
+    uint4 u = *cp;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], scale2);
+    *cp = u;
+  }
+}
+
+// XF, dW (A = dS^T: MN-major slabs of [64 tokens][64 vocabulary columns]): the
+// producer copies the 64 tokens' scales of the stage (one 256-column tile: a
+// CTA's 128 vocabulary rows lie in one) next to the stage; this many bytes.
+constexpr int kXfScaleBytes = 64 * 4;
+
 // WIDE = 1 (2-CTA pairs, store / accumulate epilogues): each work unit is a
 // 256 x 512 output tile computed as two N = 256 MMAs per K step that share the
 // A stage, so a CTA pulls 25% fewer operand bytes from L2 per MMA.  Both halves
 // fill all 512 TMEM columns, so there is a single accumulator: the next unit's
 // MMAs wait for the epilogue (worth it where units are long, as in dH).
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// XF = 1 (2-CTA pairs, bf16, store / accumulate epilogues): the A operand is a
+// stage of stored exponentials that the transform warps turn into dS.  Each
+// CTA's copies then complete on its own barriers (the transform warps of both
+// CTAs wait for them), and the MMA issuer waits for the transforms of both
+// CTAs on a third ring of barriers.
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
+__global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
+  static_assert(!XF || (PAIR && sizeof(Elem) == 2 && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
+                "operand transform: bf16 2-CTA pairs with a store or accumulate epilogue");
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
@@ -237,6 +296,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int kSlabBytes = kBKe * kRowBytes;
   constexpr uint32_t kIdesc =
       idesc_dense(ElemTraits<Elem>::kFmt, kBM * kCtas, kBN, A_MN, B_MN);
+  // copies of each CTA complete on its own barriers (else on the leader's)
+  constexpr bool kLocalCopies = XF || !PAIR;
+  // dW with the operand transform: the stage's token scales ride with the stage,
+  // in slots at the end of the barrier region
+  constexpr bool kXfW = XF && A_MN;
+  constexpr int kXfSlotOffset = 512;  // barriers and flags use less
+  static_assert(!kXfW || kXfSlotOffset + kNS * kXfScaleBytes <= kBarrierRegion, "scale slots");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -244,11 +310,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint8_t* staging = smem + kRingBytes + kBarrierRegion;  // 1024-B aligned
   uint64_t* empty_bar = full_bar + kNS;
-  uint64_t* tfull_bar = empty_bar + kNS;
+  uint64_t* ready_bar = empty_bar + kNS;  // XF: stage transformed in both CTAs
+  uint64_t* tfull_bar = ready_bar + kNS;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* issued_slot = tmem_slot + 2;  // stages whose copies this CTA's producer issued
+  float* xf_slot = reinterpret_cast<float*>(smem + kRingBytes + kXfSlotOffset);  // [kNS][64]
+  static_assert(3 * kStagesPair * 8 + 5 * 8 + 3 * 4 <= kXfSlotOffset, "barrier region");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -262,6 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&ready_bar[s], kCtas);  // one arrival per CTA (the stage's transform warp)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -269,6 +340,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *issued_slot = 0u;
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
@@ -289,7 +361,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const Ctl ctl{p.status, p.spin_limit, abort_flag};
+  const uint32_t peer_abort =
+      PAIR ? mapa_shared(const_cast<int*>(abort_flag), rank ^ 1u) : 0u;
+  const Ctl ctl{p.status, p.spin_limit, abort_flag, peer_abort};
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -311,15 +385,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* a_s = smem + s * kSBytes;
           uint8_t* b_s = a_s + kATileBytes;
-          if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
-          const uint32_t fb = PAIR ? mapa_shared(&full_bar[s], 0) : 0u;
+          if (kLocalCopies) mbar_arrive_expect_tx(&full_bar[s], kSBytes + (kXfW ? kXfScaleBytes : 0));
+          else if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
+          const uint32_t fb = kLocalCopies ? 0u : mapa_shared(&full_bar[s], 0);
           const int k0 = kb * kBKe;
+          if (kXfW)  // the stage's 64 token scales of this CTA's vocabulary tile
+            bulk_load_1d(xf_slot + s * (kXfScaleBytes / 4),
+                         p.xf_sc + static_cast<int64_t>(m0 >> 8) * p.xf_ld + k0, kXfScaleBytes,
+                         &full_bar[s]);
 #pragma unroll
           for (int sl = 0; sl < (A_MN ? kBM / kMNe : 1); ++sl) {
             void* dst = a_s + sl * kSlabBytes;
             const int x = A_MN ? m0 + sl * kMNe : k0, y = A_MN ? k0 : m0;
-            if (PAIR) tma_load_2d_pair(&tmA, fb, dst, x, y);
-            else tma_load_2d(&tmA, &full_bar[s], dst, x, y);
+            if (kLocalCopies) tma_load_2d(&tmA, &full_bar[s], dst, x, y);
+            else tma_load_2d_pair(&tmA, fb, dst, x, y);
           }
 #pragma unroll
           for (int h = 0; h < kHalves; ++h) {
@@ -328,22 +407,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
               void* dst = b_s + h * kBBytes + sl * kSlabBytes;
               const int x = B_MN ? nh + sl * kMNe : k0, y = B_MN ? k0 : nh;
-              if (PAIR) tma_load_2d_pair(&tmB, fb, dst, x, y);
-              else tma_load_2d(&tmB, &full_bar[s], dst, x, y);
+              if (kLocalCopies) tma_load_2d(&tmB, &full_bar[s], dst, x, y);
+              else tma_load_2d_pair(&tmB, fb, dst, x, y);
             }
           }
           ++issued;
         }
       }
-      if (!ok && leader) {
-        // Let the copies already issued land before the CTA exits.
-        Ctl drain{p.status, kDrainLimit, abort_flag};
-        volatile int no_abort = 0;
-        drain.abort_flag = &no_abort;
-        const uint32_t first = issued > kNS ? issued - kNS : 0;
-        for (uint32_t n = first; n < issued; ++n)
-          wait_bar(&full_bar[n % kNS], (n / kNS) & 1u, drain);
-      }
+      *issued_slot = issued;
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -364,7 +435,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           const uint32_t s = consumed % kNS;
           const uint32_t ph = (consumed / kNS) & 1u;
-          if (!wait_bar(&full_bar[s], ph, ctl, kPark)) {
+          const bool got = XF ? wait_bar(&ready_bar[s], ph, ctl, kPark)
+                              : wait_bar(&full_bar[s], ph, ctl, kPark);
+          if (!got) {
             ok = false;
             break;
           }
@@ -406,14 +479,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is released.
         volatile int no_abort = 0;
-        Ctl drain{p.status, kDrainLimit, &no_abort};
+        Ctl drain{p.status, kDrainLimit, &no_abort, 0u};
         if (PAIR) umma_commit_pair(drain_bar, 0x1);
         else umma_commit(drain_bar);
         wait_bar(drain_bar, 0, drain);
       }
     }
     __syncwarp();
-  } else {
+  } else if (XF && warp >= 6) {
+    // ------------------------------------------------------------ operand transform
+    // Transform warp xw scales this CTA's A stages n = xw, xw + 4, ... (four
+    // stages in flight), each lane four of the stage's 128 rows of 128 bytes:
+    //   dH (A = dS [rows][V], K-major): logit rows m0 + lane + 32 i, with the
+    //      stage's tile scales loaded before the stage's data is waited for;
+    //   dW (A = dS^T, slabs [64 tokens][64 columns]): token rows of the slabs,
+    //      scales from the slot the producer filled with the stage.
+    // The rows written are read only by this CTA's tensor core (each CTA of a
+    // pair supplies its own 128 rows of A), so the proxy fence and a CTA-scope
+    // release on the arrival order them before the leader issues the MMAs.
+    const int xw = warp - 6;
+    uint32_t n = 0;
+    bool ok = true;
+    for (int t = unit; t < total_tiles && ok; t += units) {
+      const UnitRange ur = unit_range(t, p);
+      int tm, tn;
+      tile_coords(ur.tile, p, tm, tn);
+      const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;
+      for (int kb = ur.kb0; kb < ur.kb1; ++kb, ++n) {
+        if (static_cast<int>(n & 3u) != xw) continue;
+        const uint32_t s = n % kNS;
+        const uint32_t ph = (n / kNS) & 1u;
+        const int k0 = kb * kBKe;
+        float sc[4];
+        if (A_MN == 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = m0 + lane + 32 * i;
+            sc[i] = row < p.xf_rows
+                        ? __ldg(p.xf_sc + static_cast<int64_t>(k0 >> 8) * p.xf_ld + row)
+                        : 0.f;
+          }
+        }
+        if (!wait_bar(&full_bar[s], ph, ctl, true)) {
+          ok = false;
+          break;
+        }
+        uint8_t* a_s = smem + s * kSBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;  // 0 .. 127
+          if (A_MN == 0) {
+            if (m0 + r < p.xf_rows)
+              xf_row(a_s + r * kRowBytes, r & 7, __float2bfloat162_rn(sc[i]));
+          } else {
+            const int kk = r & 63;
+            if (k0 + kk < p.xf_rows)
+              xf_row(a_s + (r >> 6) * kSlabBytes + kk * kRowBytes, kk & 7,
+                     __float2bfloat162_rn(xf_slot[s * (kXfScaleBytes / 4) + kk]));
+          }
+        }
+        fence_proxy_async_smem();  // generic writes -> the tensor core's reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(&ready_bar[s], 0));
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
     // Each warp stages its 32 rows x 32 columns of output in shared memory
     // (two buffers, swizzled to match the output map) and one lane issues a TMA
@@ -435,9 +566,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else mbar_arrive(&tempty_bar[buf]);
       }
     };
-    // Stage v * scale (32 values of this thread's row) and store the warp's box
-    // at output column x, output-map row y (rows past row_end are not written).
-    // (stores v * scale - shift)
+    // Stage v * scale - shift (32 values of this thread's row) and store the
+    // warp's box at output column x, output-map row y (rows past the map's
+    // extent are not written).
     auto store_box = [&](const uint32_t(&v)[32], float scale, float shift, int x, int y,
                          bool fp32_out, bool reduce, bool issue) {
       uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
@@ -509,6 +640,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
+        const int gstart = gi;  // first cached entry of this tile (for the dS transform)
         // Pass 1: the row's maximum over this tile (base-2 units) and the
         // cached entries' cross term, from the fp32 accumulator.
 #pragma unroll 1
@@ -532,12 +664,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
         }
-        // Pass 2: sum of 2^(x - max), and the stored logits shifted by the tile
-        // maximum (s~ - max): the entries that carry the probability mass sit
-        // near 0, where the stored value's rounding error vanishes.  Readers
-        // add the maximum back from the tile statistics.
-        const float shift = (p.partials != nullptr && mx > -INFINITY) ? mx * 0.6931471805599453f
-                                                                       : 0.f;
+        // Pass 2: sum of 2^(x - max) and the stored values.  STORE_SHIFTED
+        // stores s~ - max: the entries that carry the probability mass sit near
+        // 0, where the stored value's rounding error vanishes; readers add the
+        // maximum back from the tile statistics.  STORE_EXP stores the
+        // exponentials 2^(x - max) in (0, 1].
+        // Teacher-hidden student pass (tbuf given): the teacher's stored tile
+        // t~ - mt gives, per column, w = 2^((t~ - mt) log2 e) and t~ - s~; the
+        // tile's sums A = sum w (t~ - s~) and U = sum 2^(x - max) (s~ - t~) are
+        // formed here from fp32 values.
+        const bool hid = p.tbuf != nullptr && rv;
+        const float* trow = hid ? p.tbuf + static_cast<int64_t>(grow) * p.tld : nullptr;
+        const float mt = hid ? __ldg(&p.tpart[static_cast<int64_t>(grow) * p.tiles_n + tn].x) *
+                                   kLn2f
+                             : 0.f;
+        float A = 0.f, U = 0.f;
+        const float shift = (p.partials != nullptr && mx > -INFINITY) ? mx * kLn2f : 0.f;
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
           uint32_t v[32];
@@ -548,13 +690,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int cb = col0 + c * 32;
           const int nvalid = p.cols_valid - cb;
           if (nvalid <= 0) continue;
+          uint32_t e[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            se += i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
-          if (p.store) store_box(v, rscale, shift, cb, row0, kElemF32, false, warp_rows);
+          for (int i = 0; i < 32; ++i) {
+            const float x = i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
+            se += x;
+            e[i] = __float_as_uint(x);
+          }
+          if (hid) {
+            float tv[32];
+            if (nvalid >= 32) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 t4 = __ldg(reinterpret_cast<const float4*>(trow + cb) + j);
+                tv[4 * j] = t4.x;
+                tv[4 * j + 1] = t4.y;
+                tv[4 * j + 2] = t4.z;
+                tv[4 * j + 3] = t4.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) tv[i] = i < nvalid ? __ldg(trow + cb + i) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < nvalid) {
+                const float d = (tv[i] + mt) - __uint_as_float(v[i]) * rscale;  // t~ - s~
+                A = fmaf(ex2_approx(tv[i] * kLog2e), d, A);
+                U = fmaf(__uint_as_float(e[i]), -d, U);
+              }
+            }
+          }
+          if (p.store == STORE_EXP)
+            store_box(e, 1.f, 0.f, cb, row0, false, false, warp_rows);
+          else if (p.store == STORE_SHIFTED)
+            store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
         }
         if (rv && p.partials != nullptr)
-          p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
+          p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] =
+              p.tbuf != nullptr ? make_float4(mx, se, A, U)
+                                : make_float4(mx, se, cross, __int_as_float(gstart));
       } else if (EPI == EPI_DLOGITS) {
         float coef = 0.f, cm = 0.f, l2 = 0.f;
         const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
@@ -629,6 +804,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   }
 
+  // Every role of both CTAs has finished (or given up).  After an abort, copies
+  // that were issued but never consumed may still be in flight; wait for them
+  // before either CTA of the pair can exit.
+  __syncthreads();
+  if (PAIR) cluster_sync();
+  bool aborted = *abort_flag != 0;
+  if (PAIR) aborted = aborted || ld_cluster_u32(peer_abort) != 0u;
+  if (aborted && warp == 4 && lane == 0) {
+    volatile int no_abort = 0;
+    const Ctl drain{p.status, kDrainLimit, &no_abort, 0u};
+    const uint32_t mine = *issued_slot;
+    uint32_t hi = mine;
+    bool drain_here = true;
+    if (!kLocalCopies) {
+      // Both CTAs' copies complete on the leader's barriers, which the leader
+      // armed for both CTAs' bytes of every stage it issued.  Settle the stages
+      // one producer issued and the other did not, then wait for the last ring's
+      // worth of stages.
+      drain_here = leader;
+      if (leader) {
+        const uint32_t peer = ld_cluster_u32(mapa_shared(issued_slot, 1));
+        for (uint32_t n = peer; n < mine; ++n)  // the peer's bytes never come
+          mbar_complete_tx(&full_bar[n % kNS], kSBytes);
+        for (uint32_t n = mine; n < peer; ++n)  // armed for the peer's bytes only
+          mbar_arrive_expect_tx(&full_bar[n % kNS], kSBytes);
+        hi = peer > mine ? peer : mine;
+      }
+    }
+    if (drain_here) {
+      const uint32_t first = hi > kNS ? hi - kNS : 0;
+      for (uint32_t n = first; n < hi; ++n) wait_bar(&full_bar[n % kNS], (n / kNS) & 1u, drain);
+    }
+  }
   __syncthreads();
   if (PAIR) cluster_sync();  // neither CTA of a pair leaves while the other still works
   if (warp == 5) {

@@ -341,125 +341,196 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   }
 }
 
-// Two block-wide sums in a fixed order (warp shuffles, then warp 0).
-__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
-  a = warp_sum(a);
-  b = warp_sum(b);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(a, b);
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float2 v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : make_float2(0.f, 0.f);
-    v.x = warp_sum(v.x);
-    v.y = warp_sum(v.y);
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float2 r = red[0];
-  __syncthreads();
-  return r;
+// dS from the stored exponentials (bf16 top-K, fused path).  The logits pass
+// stores e_j = 2^(s~_j log2 e - M) with M the (row, 256-column tile) maximum
+// (base 2), so the dense part of dS_j = c (m p_s,j - q_j [j in S]) is
+// scale * e_j with
+//   scale = c m 2^(max(M - lse log2 e, -64)),
+// where c = g / (n T) (0 on masked rows).  The floor at 2^-64 keeps scale a
+// normal float when a tile lies far below the row's maximum; the dense part it
+// then adds, at most c m 2^-64 per entry, is far below any entry that matters.
+// The correction -c q_j at a cached column is folded into the stored value
+// itself (xf_patch_kernel), so that dS = scale * e everywhere and the gradient
+// contractions apply one factor per (row, tile) to their operand stages.
+__device__ __forceinline__ float xf_scale(float cm, float M2, float l2) {
+  return cm * ex2_approx(fmaxf(M2 - l2, -64.f));
 }
 
-// Full-vocabulary mode (one CTA per row).  A = sum_j p_t,j (t~_j - s~_j) gives the
-// forward KL A - lse_t + lse_s; with reverse weight beta > 0 also
-// u_bar = sum_j p_s,j (s~_j - t~_j), the reverse KL u_bar - lse_s + lse_t, and
+// One warp per row, lanes over the K cached entries: e_j <- e_j - c q_j / scale
+// at each cached column j of this head (bf16 stored exponentials in S, row
+// stride ld), with scale as xf_scale for j's tile.  Reads the logits pass's
+// tile maxima (part.x); masked rows and rows without cache mass keep e (their
+// scale is 0).
+__global__ void xf_patch_kernel(__nv_bfloat16* __restrict__ S, int64_t ld,
+                                const float4* __restrict__ part, int tiles_n, int rows, int V,
+                                const float* __restrict__ lse, const uint8_t* __restrict__ mask,
+                                const float2* __restrict__ rowinfo,
+                                const int* __restrict__ sidx, const float* __restrict__ sq,
+                                int K, const Scalars* sc, const float* g_dev, float g_host,
+                                float invT, const float* __restrict__ T_row) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const float c = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
+  const float cm = c * rowinfo[row].x;
+  if (cm == 0.f) return;
+  const float l2 = lse[row] * kLog2e;
+  const int* ri = sidx + static_cast<int64_t>(row) * K;
+  const float* rq = sq + static_cast<int64_t>(row) * K;
+  __nv_bfloat16* srow = S + static_cast<int64_t>(row) * ld;
+  for (int i = lane; i < K; i += 32) {
+    const int j = ri[i];  // in [0, V): a cached column of this head; else empty or elsewhere
+    if (static_cast<unsigned>(j) >= static_cast<unsigned>(V)) continue;
+    const float scale =
+        xf_scale(cm, part[static_cast<int64_t>(row) * tiles_n + (j >> 8)].x, l2);
+    srow[j] = __float2bfloat16_rn(__bfloat162float(srow[j]) - c * rq[i] / scale);
+  }
+}
+
+// Scales of dS (xf_scale) for the chunk's rows, transposed for the gradient
+// contractions: sc_out[t * ld + row] for tile t.  A block covers 32 rows (lane
+// = row, so the writes of each tile are contiguous) and its warps share the
+// tiles.
+__global__ void xf_scales_kernel(const float4* __restrict__ part, int tiles_n, int rows,
+                                 const float* __restrict__ lse, const uint8_t* __restrict__ mask,
+                                 const float2* __restrict__ rowinfo, const Scalars* sc,
+                                 const float* g_dev, float g_host, float invT,
+                                 const float* __restrict__ T_row, float* __restrict__ sc_out,
+                                 int64_t ld) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 32 + lane;
+  if (row >= rows) return;
+  const float cm = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row) * rowinfo[row].x;
+  const float l2 = lse[row] * kLog2e;
+  const float4* pr = part + static_cast<int64_t>(row) * tiles_n;
+  for (int t = warp; t < tiles_n; t += blockDim.x >> 5)
+    sc_out[static_cast<int64_t>(t) * ld + row] = xf_scale(cm, pr[t].x, l2);
+}
+
+// Teacher-hidden mode, one warp per row: from the tile statistics of the two
+// logits passes -- student (max2, sumexp2, A_tile, U_tile) and teacher (max2,
+// sumexp2, ., .), with A_tile = sum 2^(t - mt) (t~ - s~) and
+// U_tile = sum 2^(s - ms) (s~ - t~) over the tile (fp32, formed in the student
+// pass's epilogue) -- the row's
+//   lse_s, lse_t (merged over the tiles, or given: lse_s_in / lse_t_in),
+//   A = sum_j p_t,j (t~_j - s~_j) = sum_tiles 2^(mt - lse_t log2 e) A_tile,
+//   U = sum_j p_s,j (s~_j - t~_j) = sum_tiles 2^(ms - lse_s log2 e) U_tile.
+// Forward KL = A - lse_t + lse_s and reverse KL = U - lse_s + lse_t, so the row
+// loss (1 - beta) KL(p_t || p_s) + beta KL(p_s || p_t) needs no other pass.
+// Writes (each optional): lse_s_out / lse_t_out; row_loss (0 on masked rows;
+// add_lse = 0 leaves the lse terms out: a vocabulary shard's share, whose A and
+// U cover its own columns only); sums_out[row] = (A, U); ubar_out[row] = u_bar,
+// the whole-vocabulary sum p_s (s~ - t~) that the reverse-KL gradient needs --
+// U itself, or the sum of every shard's U from sums_all [P][rows][2] when given.
+// Sums run in a fixed order.
+__global__ void hidden_sums_kernel(const float4* __restrict__ part_s,
+                                   const float4* __restrict__ part_t, int tiles_n, int rows,
+                                   const float* __restrict__ lse_s_in,
+                                   const float* __restrict__ lse_t_in, float* __restrict__ lse_s_out,
+                                   float* __restrict__ lse_t_out, const uint8_t* __restrict__ mask,
+                                   float beta, int add_lse, float* __restrict__ row_loss,
+                                   float* __restrict__ sums_out, float* __restrict__ ubar_out,
+                                   const float* __restrict__ sums_all, int P) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const float4* ps = part_s + static_cast<int64_t>(row) * tiles_n;
+  const float4* pt = part_t + static_cast<int64_t>(row) * tiles_n;
+  float lse_s, lse_t;  // natural units; the weights below use them in base 2
+  if (lse_s_in != nullptr) {
+    lse_s = lse_s_in[row];
+    lse_t = lse_t_in[row];
+  } else {
+    float Ms = -INFINITY, Mt = -INFINITY;
+    for (int i = lane; i < tiles_n; i += 32) {
+      Ms = fmaxf(Ms, ps[i].x);
+      Mt = fmaxf(Mt, pt[i].x);
+    }
+    Ms = warp_max(Ms);
+    Mt = warp_max(Mt);
+    float Zs = 0.f, Zt = 0.f;
+    for (int i = lane; i < tiles_n; i += 32) {
+      Zs += ps[i].y * ex2_approx(ps[i].x - Ms);
+      Zt += pt[i].y * ex2_approx(pt[i].x - Mt);
+    }
+    // as row_reduce_kernel merges a row: the same bits as a caller-given lse
+    lse_s = (Ms + log2f(warp_sum(Zs))) * kLn2;
+    lse_t = (Mt + log2f(warp_sum(Zt))) * kLn2;
+  }
+  const float ls2 = lse_s * kLog2e, lt2 = lse_t * kLog2e;
+  float A = 0.f, U = 0.f;
+  for (int i = lane; i < tiles_n; i += 32) {
+    const float4 s = ps[i];
+    A += ex2_approx(pt[i].x - lt2) * s.z;
+    U += ex2_approx(s.x - ls2) * s.w;
+  }
+  A = warp_sum(A);
+  U = warp_sum(U);
+  if (lane == 0) {
+    if (lse_s_out != nullptr) lse_s_out[row] = lse_s;
+    if (lse_t_out != nullptr) lse_t_out[row] = lse_t;
+    if (sums_out != nullptr) {
+      sums_out[2 * row] = A;
+      sums_out[2 * row + 1] = U;
+    }
+    if (ubar_out != nullptr) {
+      float ub = U;
+      if (sums_all != nullptr) {
+        const int64_t blk = static_cast<int64_t>(rows) * 2;
+        ub = 0.f;
+        for (int q = 0; q < P; ++q) ub += sums_all[q * blk + 2 * row + 1];
+      }
+      ubar_out[row] = ub;
+    }
+    if (row_loss != nullptr) {
+      const bool keep = mask == nullptr || mask[row] != 0;
+      const float dl = add_lse ? lse_s - lse_t : 0.f;
+      row_loss[row] = keep ? (1.f - beta) * (A + dl) + beta * (U - dl) : 0.f;
+    }
+  }
+}
+
+// Full-vocabulary mode, dS in place over the student buffer (one CTA per row):
 //   dS = c [(1 - beta)(p_s - p_t) + beta p_s (u - u_bar)],  u = s~ - t~,
-// written in place over S in a second pass (u_bar is needed first).  With
-// beta = 0 the single pass writes dS = c (p_s - p_t).
-// phase: kDlfBoth does the above; for a vocabulary shard with beta > 0 the
-// two passes are split around an exchange: kDlfSums writes this shard's
-// (A, U) to sums_out[row] and nothing else, and kDlfGrad reads every shard's
-// (A, U) from sums_all ([P][rows][2], rank order), takes u_bar as the sum of
-// the U and runs only the second pass (the row loss from this shard's A, U).
-constexpr int kDlfBoth = 0;
-constexpr int kDlfSums = 1;
-constexpr int kDlfGrad = 2;
+// c = g / (n T) (0 on masked rows), with p_s from the stored s~ - ms (element
+// type of H), p_t from the stored t~ - mt (fp32), the tile maxima (base 2)
+// from the two passes' statistics, the row lse's and u_bar per row.  Columns
+// from V to the row's padded end are written as 0.
 template <typename Elem>
-__global__ void dlogits_full_kernel(Elem* __restrict__ S, const Elem* __restrict__ Tt, int64_t ld,
+__global__ void dlogits_full_kernel(Elem* __restrict__ S, const float* __restrict__ Tt, int64_t ld,
                                     int V, const float* __restrict__ lse_s,
                                     const float* __restrict__ lse_t,
+                                    const float* __restrict__ ubar,
                                     const uint8_t* __restrict__ mask, const Scalars* sc,
                                     const float* g_dev, float g_host, float invT,
-                                    const float* __restrict__ T_row,
-                                    float* __restrict__ row_loss, int write_grad, float beta,
+                                    const float* __restrict__ T_row, float beta,
                                     const float4* __restrict__ part_s,
-                                    const float4* __restrict__ part_t, int tiles_n,
-                                    int add_lse, int phase, float* __restrict__ sums_out,
-                                    const float* __restrict__ sums_all, int P, int rank,
-                                    int rows) {
-  __shared__ float2 red[32];
+                                    const float4* __restrict__ part_t, int tiles_n) {
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
-  const Elem* trow = Tt + static_cast<int64_t>(row) * ld;
+  const float* trow = Tt + static_cast<int64_t>(row) * ld;
   const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
   const float ls2 = lse_s[row] * kLog2e, lt2 = lse_t[row] * kLog2e;
+  const float cf = coef * (1.f - beta), cr = coef * beta;
+  const float ub = beta > 0.f ? ubar[row] : 0.f;
   const int nvec = (V + 7) >> 3;
-  const bool single = beta == 0.f;
-  float A = 0.f, U = 0.f;
-  for (int v = (phase == kDlfGrad ? nvec : 0) + threadIdx.x; v < nvec; v += blockDim.x) {
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float fs[8], ft[8];
     load8<Elem>(srow + v * 8, fs);
-    load8<Elem>(trow + v * 8, ft);
-    // stored values are shifted by their tile maxima (8 | 256: one tile per vector)
-    const float ms2 = tile_max2(part_s, row, tiles_n, v * 8);
-    const float mt2 = tile_max2(part_t, row, tiles_n, v * 8);
-    const float dshift = (mt2 - ms2) * kLn2;  // (t~ - s~) = (ft - fs) + dshift
+    load8<float>(trow + v * 8, ft);
+    // 8 | 256: the vector lies in one tile
+    const float ms2 = part_s[static_cast<int64_t>(row) * tiles_n + (v >> 5)].x;
+    const float mt2 = part_t[static_cast<int64_t>(row) * tiles_n + (v >> 5)].x;
+    const float dshift = (ms2 - mt2) * kLn2;  // (s~ - t~) = (fs - ft) + dshift
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const bool in = v * 8 + i < V;
       const float pt = ex2_approx(fmaf(ft[i], kLog2e, mt2 - lt2));
       const float ps = ex2_approx(fmaf(fs[i], kLog2e, ms2 - ls2));
-      const float u = (fs[i] - ft[i]) - dshift;  // s~ - t~
-      A -= in ? pt * u : 0.f;
-      U += in ? ps * u : 0.f;
-      fs[i] = in ? operand_round<Elem>(coef * (ps - pt)) : 0.f;
+      const float g = cf * (ps - pt) + cr * ps * (((fs[i] - ft[i]) + dshift) - ub);
+      fs[i] = in ? operand_round<Elem>(g) : 0.f;
     }
-    if (write_grad && single) store8<Elem>(srow + v * 8, fs);
-  }
-  float2 r;
-  float ubar;
-  if (phase == kDlfGrad) {  // every shard's sums, merged in rank order
-    const int64_t blk = static_cast<int64_t>(rows) * 2;
-    r = make_float2(sums_all[rank * blk + 2 * row], sums_all[rank * blk + 2 * row + 1]);
-    ubar = 0.f;
-    for (int q = 0; q < P; ++q) ubar += sums_all[q * blk + 2 * row + 1];
-  } else {
-    r = block_sum2(A, U, red);
-    ubar = r.y;
-  }
-  if (phase == kDlfSums) {
-    if (threadIdx.x == 0) {
-      sums_out[2 * row] = r.x;
-      sums_out[2 * row + 1] = r.y;
-    }
-    return;
-  }
-  if (write_grad && !single) {
-    const float cf = coef * (1.f - beta), cr = coef * beta;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-      float fs[8], ft[8];
-      load8<Elem>(srow + v * 8, fs);
-      load8<Elem>(trow + v * 8, ft);
-      const float ms2 = tile_max2(part_s, row, tiles_n, v * 8);
-      const float mt2 = tile_max2(part_t, row, tiles_n, v * 8);
-      const float dshift = (mt2 - ms2) * kLn2;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool in = v * 8 + i < V;
-        const float pt = ex2_approx(fmaf(ft[i], kLog2e, mt2 - lt2));
-        const float ps = ex2_approx(fmaf(fs[i], kLog2e, ms2 - ls2));
-        const float g = cf * (ps - pt) + cr * ps * (((fs[i] - ft[i]) - dshift) - ubar);
-        fs[i] = in ? operand_round<Elem>(g) : 0.f;
-      }
-      store8<Elem>(srow + v * 8, fs);
-    }
-  }
-  if (threadIdx.x == 0 && row_loss != nullptr) {
-    const bool keep = mask == nullptr || mask[row] != 0;
-    // add_lse = 0: a vocabulary shard's share, the sums over its columns only
-    const float dl = add_lse ? lse_s[row] - lse_t[row] : 0.f;
-    const float fwd = r.x + dl;
-    const float rev = r.y - dl;
-    row_loss[row] = keep ? (1.f - beta) * fwd + beta * rev : 0.f;
+    store8<Elem>(srow + v * 8, fs);
   }
 }
 

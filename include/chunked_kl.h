@@ -184,9 +184,12 @@ int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss,
  * Errors: KL_ERR_DTYPE unless bf16 + KL_TEACHER_TOPK; KL_ERR_TOO_LARGE when a
  * single token row of scratch (16 * ceil(V / 256) + 8 * K + 8 bytes, plus a
  * 256-byte header) exceeds KL_NOALLOC_SCRATCH_BYTES; the other codes as kl_fwd.
- * It calls no cudaMalloc, cudaFree or other allocating routine.  The first call
- * on a device looks up the scratch array's device address (cudaGetSymbolAddress,
- * with that device current); make that first call before any stream capture.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.  Every call
+ * looks up the scratch array's device address for the current device and
+ * context (cudaGetSymbolAddress, with that device current), so the address
+ * stays right after a context is destroyed and created again; the first call on
+ * a device may also load the library's kernels, so make it before any stream
+ * capture.
  * All calls share the one array and it keeps the last call's contents (each
  * call re-initialises what it reads), so calls whose kernels overlap on the GPU
  * (different streams, or different host threads) race: order them. */

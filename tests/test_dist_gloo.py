@@ -83,3 +83,39 @@ def test_two_rank_shards_with_global_normalizer_match_single_process():
     assert loss == pytest.approx(ref, rel=1e-12)
     assert dw_err < 1e-12
     assert slowest == 2.0
+
+
+def _reduce_worker(rank, world, port, q):
+    from chunked_kl_loss_tma_b200.dist import dW_shard_rows, reduce_scatter_rows, sum_over_ranks
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        V, d = 11, 3  # V not a multiple of the world size: the last block is short
+        parts = [torch.arange(V * d, dtype=torch.float32).reshape(V, d) * (r + 1)
+                 for r in range(world)]
+        total = sum(parts)
+        t = parts[rank].clone()
+        sum_over_ranks(t)
+        shard = reduce_scatter_rows(parts[rank].clone())
+        a, b = dW_shard_rows(V, world, rank)
+        q.put((rank, torch.equal(t, total), torch.equal(shard, total[a:b]), (a, b)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_sum_and_reduce_scatter_helpers():
+    """sum_over_ranks and reduce_scatter_rows (the head-gradient reductions of
+    the token data-parallel form) over gloo, against the plain sums."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_reduce_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(r[1] and r[2] for r in res), res
+    assert [r[3] for r in res] == [(0, 6), (6, 11)]

@@ -5,12 +5,16 @@ dH), against the fp64 oracle.
 Outputs the oracle can compute one by one are compared element by element on
 sampled rows (first and last rows, chunk boundaries, masked rows, random
 rows): row loss, lse and dH rows, each sampled row evaluated by the oracle as a
-problem of its own with the full problem's normaliser.  At N=4096 the oracle
-also makes its full pass (every row's lse), which gives the loss itself and
-sampled rows of dW.  Elsewhere dW is checked through identities that hold at
-any size: every dS row sums to zero (sum_j (m p_s,j - q_j) = m - m = 0, and
-sum_j (p_s,j - p_t,j) = 0), so sum_j dW_j = 0; and <dW, W> = <dH, H> =
-sum_{n,j} dS_nj s_nj.
+problem of its own with the full problem's normaliser.  Up to N=65536 the
+oracle also makes its full pass over every row, which gives the loss itself,
+every row's loss, and dW on sampled vocabulary rows -- among them the rows the
+teacher's mass concentrates on (the most frequent cached ids, or the teacher's
+most frequent argmax in the teacher-hidden mode).  At N=262144, where a full
+fp64 pass takes too long, the loss is checked as the mean of the row losses and
+dW through identities that hold at any size: every dS row sums to zero
+(sum_j (m p_s,j - q_j) = m - m = 0, and sum_j (p_s,j - p_t,j) = 0), so
+sum_j dW_j = 0; and <dW, W> = <dH, H> = sum_{n,j} dS_nj s_nj.  The identities
+are checked everywhere as extra checks.
 
 Tolerances as in test_parity_gpu.py: loss relative error <= 1e-3; gradient
 max-abs error <= 2e-2 * max|oracle gradient| (over the sampled entries)."""
@@ -84,6 +88,45 @@ def _identities(w, out):
     assert abs(a) > 0
 
 
+def _vocab_rows(w, n_hot=24, n_random=16, seed=1):
+    """Vocabulary rows for the dW check: the ids that carry the teacher's mass
+    most often (the cached ids, or the teacher's argmax computed with a plain
+    torch matmul), random rows, and the first and last rows."""
+    if w.mode == "topk":
+        ids = w.topk_idx[:, :4].reshape(-1)
+        ids = ids[ids >= 0]
+    else:
+        ids = torch.cat([(w.Ht[i:i + 2048].float() @ w.Wt.float().T).argmax(1)
+                         for i in range(0, w.N, 2048)])
+    counts = torch.bincount(ids.long(), minlength=w.V)
+    hot = torch.topk(counts, n_hot).indices.cpu().numpy()
+    rnd = np.random.default_rng(seed).choice(w.V, n_random, replace=False)
+    return np.unique(np.concatenate([hot, rnd, [0, w.V - 1]]))
+
+
+def _full_oracle_pass(w, out, n_valid, reverse_weight=0.0):
+    """The oracle over every row: the loss (relative error <= 1e-3), every
+    row's loss, and dW on sampled vocabulary rows (max-abs error <= 2e-2 of the
+    largest oracle entry)."""
+    vrows = _vocab_rows(w)
+    args = dict(T=w.T, mode=w.mode, mask=w.mask, want_dH=False, vocab_rows=vrows,
+                reverse_weight=reverse_weight)
+    if w.mode == "topk":
+        args.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        args.update(Ht=w.Ht, Wt=w.Wt)
+    ref = oracle.kl_loss(w.H, w.W, **args)
+    assert ref["n_valid"] == n_valid
+    assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]), \
+        (out["loss"].item(), ref["loss"])
+    rl = out["row_loss"].double().cpu().numpy()
+    assert np.max(np.abs(rl - ref["row_loss"])) <= 2e-3 * np.max(np.abs(ref["row_loss"]))
+    dW = out["dW"][torch.as_tensor(vrows, device=out["dW"].device)].double().cpu().numpy()
+    err = np.max(np.abs(dW - ref["dW"]))
+    assert err <= 2e-2 * np.max(np.abs(ref["dW"])), f"dW rows: {err}"
+    return ref
+
+
 def _loss_is_mean_of_rows(out, n_valid):
     mean = out["row_loss"].double().sum().item() / n_valid
     assert abs(out["loss"].item() - mean) <= 1e-5 * abs(mean)
@@ -97,20 +140,7 @@ def test_offline_topk_4096_full_oracle_pass():
     rows = _rows(w.N, None)
     _check_rows(w, out, rows, n_valid)
     _loss_is_mean_of_rows(out, n_valid)
-    # Full oracle pass: the loss over all rows and sampled dW rows (including
-    # rows the cache hits).
-    hits = np.unique(w.topk_idx[:64, :4].cpu().numpy())[:16]
-    vrows = np.unique(np.concatenate([hits, np.random.default_rng(1).choice(w.V, 16,
-                                                                              replace=False),
-                                      [0, w.V - 1]]))
-    ref = oracle.kl_loss(w.H, w.W, T=w.T, mode="topk", topk_idx=w.topk_idx,
-                         topk_logit=w.topk_logit, teacher_lse=w.teacher_lse, want_dH=False,
-                         vocab_rows=vrows)
-    assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"])
-    np.testing.assert_allclose(out["row_loss"].double().cpu().numpy(), ref["row_loss"],
-                               rtol=5e-3, atol=2e-3 * np.max(np.abs(ref["row_loss"])))
-    dW = out["dW"][torch.as_tensor(vrows, device="cuda")].double().cpu().numpy()
-    assert np.max(np.abs(dW - ref["dW"])) <= 2e-2 * np.max(np.abs(ref["dW"]))
+    _full_oracle_pass(w, out, n_valid)
     _identities(w, out)
 
 
@@ -141,6 +171,7 @@ def test_full_vocab_8192_teacher_hidden():
     rows = _rows(w.N, None, n_random=16)
     _check_rows(w, out, rows, w.N)
     _loss_is_mean_of_rows(out, w.N)
+    _full_oracle_pass(w, out, w.N)
     _identities(w, out)
     # the split forward gives the same loss and the teacher lse of the oracle
     f = ops.kl_fwd(w.H, w.W, **_kw(w))
@@ -176,6 +207,7 @@ def test_packed_long_32768_masked():
     rows = _rows(w.N, w.mask)
     _check_rows(w, out, rows, n_valid)
     _loss_is_mean_of_rows(out, n_valid)
+    _full_oracle_pass(w, out, n_valid)
     _identities(w, out)
 
 
@@ -203,6 +235,8 @@ def test_scaling_sweep_rows_and_flat_memory(N):
     rows = _rows(N, None, n_random=12, seed=N)
     _check_rows(w, out, rows, N)
     _loss_is_mean_of_rows(out, N)
+    if N <= 65536:
+        _full_oracle_pass(w, out, N)
     _identities(w, out)
 
 

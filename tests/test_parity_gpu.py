@@ -232,7 +232,9 @@ def test_launch_counter_and_profile():
     ops.kl_fwd_bwd(w.H, w.W, **_kw(w, chunk=128))
     prof = L.kl_profile_end()
     names = {p["name"] for p in prof}
-    assert {"gemm_logits_stats", "gemm_dH", "gemm_dW", "dlogits_topk"} <= names
+    # bf16 top-K: dS is formed inside the gradient contractions (no dlogits pass)
+    assert {"gemm_logits_stats", "xf_scales", "gemm_dH", "gemm_dW"} <= names
+    assert "dlogits_topk" not in names
     assert L.kl_launch_count() - before == sum(p["launches"] for p in prof)
     assert all(p["total_ms"] > 0 for p in prof)
 
@@ -353,39 +355,14 @@ def test_split_backward_accumulates_into_dW():
     _check_grad(b["dW"] - base, ref["dW"], "accumulated dW (split)")
 
 
-def _bf16_storage_bound(w, dtype):
-    """Teacher-hidden mode with bf16 inputs forms the loss term
-    sum_j p_t,j (t~_j - s~_j) from the stored bf16 logits, each shifted by its
-    (row, 256-column tile) maximum, so every stored value carries a rounding
-    error of at most 2^-9 |x - m|.  To first order the row loss moves by at most
-    2^-9 sum_j p_t,j (|t~_j - m_t| (1 + |t~_j - s~_j|) + |s~_j - m_s|).  Over a
-    large vocabulary these errors average out far below the 1e-3 loss target;
-    with a handful of classes they need not, so the smallest-vocabulary cases
-    are held to this bound on top of the target.  0 for fp32 inputs (fp32
-    storage)."""
-    if dtype != torch.bfloat16:
-        return 0.0
-    H, W = w.H.double().cpu().numpy(), w.W.double().cpu().numpy()
-    Ht, Wt = w.Ht.double().cpu().numpy(), w.Wt.double().cpu().numpy()
-    s, t = H @ W.T / w.T, Ht @ Wt.T / w.T
-    b = 0.0
-    for j0 in range(0, s.shape[1], 256):  # tile maxima
-        st, tt = s[:, j0:j0 + 256], t[:, j0:j0 + 256]
-        pt = np.exp(tt - np.log(np.exp(t - t.max(1, keepdims=True)).sum(1, keepdims=True))
-                    - t.max(1, keepdims=True))
-        dt = np.abs(tt - tt.max(1, keepdims=True))
-        ds = np.abs(st - st.max(1, keepdims=True))
-        b += np.sum(pt * (dt * (1 + np.abs(tt - st)) + ds))
-    return 2.0 ** -9 * b / s.shape[0]
-
-
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("N,d,V,K", [(1, 8, 1, 1), (3, 8, 7, 2), (5, 16, 9, 9), (2, 8, 300, 1)])
 def test_smallest_shapes(dtype, N, d, V, K):
     """One-row, one-class and sub-vector vocabularies (V < 8 pads the logit
     rows), the narrowest width d = 8 and a single cached entry, both teacher
     modes.  With V = 1 both distributions are a point mass: loss 0 up to
-    rounding."""
+    rounding, so the loss is held to 1e-3 relative plus an absolute 1e-6 that
+    only matters when the oracle's loss is itself zero."""
     w = wl.make_topk("tiny_shapes", N=N, d=d, V=V, K=K, d_t=8, T=1.1, dtype=dtype,
                      w_std=0.3, tw_std=0.3, seed=50 + V).to("cuda")
     for partial in (True, False):
@@ -395,7 +372,7 @@ def test_smallest_shapes(dtype, N, d, V, K):
         out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **kw)
         assert ops.status(out["workspace"]) == 0
         ref = _oracle(w, teacher_lse=kw["teacher_lse"])
-        assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-5
+        assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-6
         for k in ("dH", "dW"):
             got = out[k].double().cpu().numpy()
             assert np.max(np.abs(got - ref[k])) <= GRAD_FRAC * np.max(np.abs(ref[k])) + 1e-6, k
@@ -403,8 +380,7 @@ def test_smallest_shapes(dtype, N, d, V, K):
                        tw_std=0.3, seed=60 + V).to("cuda")
     out = ops.kl_fwd_bwd(h.H, h.W, want_row_loss=True, **_kw(h))
     ref = _oracle(h)
-    assert abs(out["loss"].item() - ref["loss"]) <= \
-        1e-3 * abs(ref["loss"]) + 1e-5 + _bf16_storage_bound(h, dtype)
+    assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-6
     for k in ("dH", "dW"):
         got = out[k].double().cpu().numpy()
         assert np.max(np.abs(got - ref[k])) <= GRAD_FRAC * np.max(np.abs(ref[k])) + 1e-6, k
