@@ -4,14 +4,16 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kernels|reference]
 
 One step = one kl_fwd_bwd call (top-K prep, logits + split-V statistics with the
-fused cache gather, row merge, dlogits, dH and dW contractions, loss mean) over
-one batch of the offline top-K workload: N=4096 tokens, d=3072, V=128256, bf16,
-teacher cache K=64 (int32 ids + fp32 logits + fp32 teacher log-sum-exp, partial
-mass kept), T=1.  Inputs are synthetic and seeded; W (0.79 GB) and the logit
-chunk (1.05 GB) are larger than the 126 MB L2, so no flush is needed between
-steps.  With --gpus N (under torchrun) every rank runs its own N=4096-token
-shard with no collective on the data path (weak scaling); the elapsed time is
-the max over ranks.
+fused cache gather, row merge, dS factors, dH and dW contractions that form dS
+from the stored exponentials, loss mean) over one batch of the offline top-K
+workload: N=4096 tokens, d=3072, V=128256, bf16, teacher cache K=64 (int32 ids +
+fp32 logits + fp32 teacher log-sum-exp, partial mass kept), T=1.  Inputs are
+synthetic and seeded; W (0.79 GB) and the logit chunk (1.05 GB) are larger than
+the 126 MB L2, so no flush is needed between steps.  With --gpus N (under
+torchrun) every rank runs its own N=4096-token shard, scaled by the global
+count of valid tokens, and each step ends with the head gradient reduce-
+scattered (or all-reduced, --dp-sync) and the loss all-reduced over NCCL (weak
+scaling); the elapsed time is the max over ranks.
 
 Prints ONE JSON line on rank 0.  `--impl reference` times the fp64 CPU oracle
 instead, on the host cores, on a bounded row sample of the same workload.
@@ -45,6 +47,8 @@ def parse():
     ap.add_argument("--workload", default="offline_topk",
                     choices=["offline_topk", "full_vocab", "packed_long", "scaling"])
     ap.add_argument("--N", type=int, default=0, help="tokens per GPU (0 = the workload's own)")
+    ap.add_argument("--d", type=int, default=0,
+                    help="offline top-K workload: student width (0 = the workload's 3072)")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--reverse-weight", type=float, default=0.0,
                     help="teacher-hidden workload: weight of the reverse KL (0 = forward KL)")
@@ -56,6 +60,12 @@ def parse():
                          "vocab: the head split by vocabulary rows over the ranks, the same "
                          "tokens on every rank, one statistics all-gather per chunk (two with "
                          "a reverse-KL weight) and an all-reduce of dH (strong scaling)")
+    ap.add_argument("--dp-sync", default="reduce_scatter",
+                    choices=["reduce_scatter", "all_reduce", "none"],
+                    help="token shards on N>1 ranks: how each step combines the head gradient "
+                         "(dW reduce-scattered into row blocks, as a sharded optimizer keeps it, "
+                         "or all-reduced; the loss shares are all-reduced) -- 'none' times the "
+                         "shards alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample", type=int, default=0,
@@ -77,7 +87,7 @@ WORKLOADS = {
 def make_workload(wl, args, dev, rank):
     seed_shift = rank * 1000
     if args.workload == "offline_topk":
-        return wl.offline_topk(device=dev, N=args.N or 4096, seed=1 + seed_shift)
+        return wl.offline_topk(device=dev, N=args.N or 4096, seed=1 + seed_shift, d=args.d or 3072)
     if args.workload == "full_vocab":
         return wl.full_vocab(device=dev, N=args.N or 8192, seed=2 + seed_shift)
     if args.workload == "packed_long":
@@ -213,6 +223,7 @@ def gpu_arm(args):
     if args.reverse_weight > 0:
         kw["reverse_weight"] = args.reverse_weight
     shard = None
+    dp_sync = args.dp_sync if (ws > 1 and not vocab) else "none"
     if vocab:
         from chunked_kl_loss_tma_b200 import vocab_parallel as vpm
 
@@ -223,6 +234,12 @@ def gpu_arm(args):
         prob, keep = ops.make_problem(w.H, W_head, v_begin=v0, V_total=w.V, **kw)
     else:
         W_head = w.W
+        if dp_sync != "none":
+            # every rank scales by the batch's global count of valid tokens
+            from chunked_kl_loss_tma_b200.dist import global_valid_count
+
+            local = w.N if w.mask is None else int(w.mask.sum().item())
+            kw["normalizer"] = float(global_valid_count(local))
         prob, keep = ops.make_problem(w.H, w.W, **kw)
     ws_bytes = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
     loss = torch.empty((), dtype=torch.float32, device=dev)
@@ -249,6 +266,17 @@ def gpu_arm(args):
         lse_t = torch.empty(w.N, dtype=torch.float32, device=dev) if w.mode == "hidden" else None
         g_one = torch.ones((), dtype=torch.float32, device=dev)
 
+    def dp_reduce():
+        """Token shards: sum the head gradient over the ranks (reduce-scatter or
+        all-reduce) and the loss shares."""
+        from chunked_kl_loss_tma_b200.dist import reduce_scatter_rows, sum_over_ranks
+
+        if dp_sync == "all_reduce":
+            sum_over_ranks(dW)
+        else:
+            reduce_scatter_rows(dW)
+        sum_over_ranks(loss.view(1))
+
     def step():
         if shard is not None:
             vpm.run_pass(shard, comm)
@@ -263,6 +291,8 @@ def gpu_arm(args):
             return
         _lib.check(_lib.kl_fwd_bwd(prob, workspace.data_ptr(), ws_bytes, 1.0, loss.data_ptr(),
                                    None, dH.data_ptr(), dW.data_ptr(), 0, stream), "kl_fwd_bwd")
+        if dp_sync != "none":
+            dp_reduce()
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -333,6 +363,8 @@ def gpu_arm(args):
                                            loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(),
                                            0, stream), "kl_fwd_bwd")
                 stager.release(slot, cstream)
+                if dp_sync != "none":
+                    dp_reduce()
                 hloss[i].copy_(loss, non_blocking=True)
                 slot = nxt
 
@@ -408,7 +440,10 @@ def gpu_arm(args):
                    "parallelism": (f"vocabulary-parallel head shards x{ws}: all-gather of row "
                                    "statistics per chunk, all-reduce of fp32 dH"
                                    if vocab else
-                                   f"weak-scaling token shards x{ws}, no data-path collective")},
+                                   f"weak-scaling token shards x{ws}, no data-path collective"
+                                   if dp_sync == "none" else
+                                   f"weak-scaling token shards x{ws}; per step the dW "
+                                   f"{dp_sync.replace('_', '-')} and a loss all-reduce (NCCL)")},
         "entry": "kl_fwd_bwd" if args.entry == "fused" else "kl_fwd + kl_bwd (recompute)",
         "step_ms_median": round(per_step[len(per_step) // 2], 4),
         "step_ms_p10_p90": [round(per_step[len(per_step) // 10], 4),
@@ -427,6 +462,8 @@ def gpu_arm(args):
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
     if args.workload != "offline_topk":
         line["metric"] = METRIC + f" [{args.workload}]"
+    elif args.d and args.d != 3072:
+        line["metric"] = METRIC + f" [d={args.d}]"
     if args.reverse_weight > 0:
         line["metric"] += f" [reverse KL weight {args.reverse_weight}]"
         line["config"]["reverse_weight"] = args.reverse_weight

@@ -6,18 +6,24 @@
 // KL": the output projection is fused into the loss, each logit chunk is
 // transient, and backward recomputes one projection per chunk).
 //
-// Per chunk of C token rows (fwd_bwd, top-K):
+// Per chunk of C token rows (fwd_bwd, top-K, bf16):
 //   prep_topk      cache -> sorted ids + teacher probabilities q, m, sum q log q
-//   gemm STATS     S~ = H_c W^T / T  (tcgen05), split-V row statistics + gather
+//   gemm STATS     S~ = H_c W^T / T  (tcgen05), split-V row statistics + gather,
+//                  stores e = 2^(s~ log2 e - tile max)
 //   row_reduce     lse_s, row loss
-//   dlogits_topk   S~ -> dS in place
-//   gemm ACCUM     dH_c = dS W: wide 256 x 512 tiles, split-K fp32 parts
+//   xf_patch       -c q folded into e at the cached columns
+//   xf_scales      per (tile, row) scale with dS = scale * e
+//   gemm ACCUM     dH_c = dS W: wide 256 x 512 tiles, split-K fp32 parts, dS
+//                  formed from e in shared memory by the transform warps
 //   splitk_reduce  the parts summed in a fixed order -> dH_c
-//   gemm ACCUM     dW (+)= dS^T H_c
-// then finalize_loss (masked mean).  No host synchronisation anywhere.  The
-// teacher-hidden mode launches the STATS GEMM twice (student, teacher) and
-// dlogits_full instead of prep_topk / dlogits_topk; the vocabulary-parallel
-// calls (kl_vp_*) split the same sequence around per-chunk exchanges.
+//   gemm ACCUM     dW (+)= dS^T H_c, dS formed the same way
+// then finalize_loss (masked mean).  No host synchronisation anywhere.  fp32
+// inputs store s~ - tile max and turn it into dS with the dlogits_topk pass.
+// The teacher-hidden mode runs the teacher pass (fp32 t~ - tile max) and then
+// the student pass, whose epilogue forms the per-tile loss sums against the
+// teacher tile; hidden_sums merges them into lse_s, lse_t, the row loss and
+// u_bar, and dlogits_full writes dS.  The vocabulary-parallel calls (kl_vp_*)
+// split the same sequence around per-chunk exchanges.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -210,6 +216,7 @@ struct Plan {
   bool xf = false;
   int64_t Cx = 0;          // (xf) row stride of the transposed dS scales: C rounded up to 64
   size_t off_xsc = 0;      // (xf) dS scales [tiles_v][Cx] fp32
+  size_t off_dsbuf = 0;    // (xf) dS chunk [C][Vp] bf16
   size_t off_ubar = 0;     // (hidden) u_bar per chunk row
   int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
   size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
@@ -327,6 +334,7 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (pl.xf && entry == KL_ENTRY_FWD_BWD) {
     pl.Cx = cdiv(pl.C, 64) * 64;
     pl.off_xsc = take(static_cast<size_t>(pl.tiles_v) * pl.Cx * 4);
+    pl.off_dsbuf = take(buf);  // dS chunk, formed by the dH contraction for dW
   }
   if (!pl.hidden) {
     pl.off_sidx = take(static_cast<size_t>(pl.C) * p->K * 4);
@@ -365,7 +373,8 @@ Plan make_plan(const kl_problem* p, int entry) {
 // ------------------------------------------------------------------ launches
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
-                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
+                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops,
+                const CUtensorMap* md = nullptr) {
   auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
@@ -396,7 +405,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md != nullptr ? *md : mc, gp);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
@@ -601,8 +610,9 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
 // dH_c = dS . W and dW (+)= dS^T . H_c for chunk rows [c0, c0 + Cn) from the
 // chunk buffer dS.  dH_f32: write dH as fp32 (a vocabulary shard's partial sum)
 // whatever Elem is.  XF = 1: the buffer holds the logits pass's exponentials,
-// patched at the cached columns (xf_patch_kernel), and the two contractions
-// form dS = scale * e in shared memory with the per-(tile, row) scales xf_sc.
+// patched at the cached columns (xf_patch_kernel); the dH contraction forms
+// dS = scale * e in shared memory with the per-(tile, row) scales xf_sc and
+// stores it to the workspace's dS chunk, which the dW contraction reads.
 template <typename Elem, int XF>
 int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
                     bool dH_f32, const float* xf_sc) {
@@ -611,11 +621,15 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
   constexpr int kMNe = kRowBytes / sizeof(Elem);
   const int64_t d = p->d;
   const uint64_t ldS = c.pl.Vp * sizeof(Elem);
+  Elem* dS_formed = XF ? reinterpret_cast<Elem*>(c.ws + c.pl.off_dsbuf) : dS;
+  CUtensorMap md;  // XF: the dS chunk written by the dH contraction, 64 x 32 boxes
+  if (XF && !make_map(&md, dS_formed, p->dtype, p->V, Cn, ldS, kBKe, 32)) return KL_ERR_CUDA;
   auto set_xf = [&](GemmParams& gp) {
     if (!XF) return;
     gp.xf_sc = xf_sc;
     gp.xf_ld = c.pl.Cx;
     gp.xf_rows = static_cast<int>(Cn);
+    gp.xf_store = 1;
   };
   // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.  When the
   // output has too few tiles to fill the GPU, V is split into ksplit parts whose
@@ -650,7 +664,8 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
       if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
         return KL_ERR_CUDA;
       KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d)));
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
       LaunchScope ls("splitk_reduce", c.st, 0,
                      (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
       if (dH_f32)
@@ -667,21 +682,23 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
       if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
         return KL_ERR_CUDA;
       KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d)));
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
                         d * sizeof(Elem)))
         return KL_ERR_CUDA;
       KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d)));
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
     }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
   {
     CUtensorMap ma, mb, mc;
     const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * d * sizeof(Elem);
-    if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
+    if (!make_map(&ma, dS_formed, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
         !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe) ||
         !make_out_map(&mc, dW, KL_DTYPE_F32, d, p->V, d * 4))
       return KL_ERR_CUDA;
@@ -695,9 +712,8 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
     gp.beta = beta;
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    set_xf(gp);
-    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1, 0, XF>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
-                                                         2.0 * Cn * p->V * d)));
+    KL_TRY((launch_gemm<Elem, 1, 1, EPI_ACCUM, 1>("gemm_dW", c.st, c.sms, ma, mb, mc, gp,
+                                                  2.0 * Cn * p->V * d)));
   }
   return KL_OK;
 }

@@ -39,10 +39,12 @@
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
 //   warp 5     TMEM allocator + MMA issuer (one thread);
-//   warps 6-9  (XF = 1 only) operand transform: turn the A stage -- the
+//   warps 6-9  (XF = 1 only, dH) operand transform: turn the A stage -- the
 //              stored exponentials e = 2^(s~ log2 e - tile max) of a logit
-//              chunk -- into dS = scale(row, tile) * e - c q at the cached
-//              entries, in shared memory, before the MMAs read it.  This is
+//              chunk, already corrected at the cached entries -- into
+//              dS = scale(row, tile) * e in shared memory before the MMAs read
+//              it, and (units of output column tile 0) store the formed stage
+//              as the dS chunk that the dW contraction then reads.  This is
 //              the dlogits step of the loss without its own pass over HBM.
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
@@ -75,7 +77,7 @@ constexpr int kGemmThreads = 192;
 constexpr int kGemmThreadsXf = 320;  // + four operand-transform warps
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kRingBytes = kStages * kStageBytes;          // 192 KB operand ring
-constexpr int kBarrierRegion = 2048;                        // barriers, TMEM slot, flags, slots
+constexpr int kBarrierRegion = 1024;                        // barriers, TMEM slot, flags
 constexpr int kStageOutBytes = 4096;                        // one 32 x 32 fp32 output box
 constexpr int kStagingBytes = 4 * 2 * kStageOutBytes;       // 4 epilogue warps x 2 buffers
 constexpr int kGemmSmemBytes = 1024 /*align*/ + kRingBytes + kBarrierRegion + kStagingBytes;
@@ -120,6 +122,8 @@ struct GemmParams {
   const float* xf_sc;
   int64_t xf_ld;
   int xf_rows;         // logit rows (tokens) that exist
+  int xf_store;        // XF: the units of output column tile 0 store each formed
+                       // dS stage through the fourth map (the dS chunk for dW)
   // DLOGITS: per-row lse (natural units), (m, .) per row, mask, and the scalars
   // of c = g / (n T): the loss normaliser n, and g (device pointer or value)
   const float* lse;
@@ -249,30 +253,28 @@ __device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 sca
   }
 }
 
-// XF, dW (A = dS^T: MN-major slabs of [64 tokens][64 vocabulary columns]): the
-// producer copies the 64 tokens' scales of the stage (one 256-column tile: a
-// CTA's 128 vocabulary rows lie in one) next to the stage; this many bytes.
-constexpr int kXfScaleBytes = 64 * 4;
-
 // WIDE = 1 (2-CTA pairs, store / accumulate epilogues): each work unit is a
 // 256 x 512 output tile computed as two N = 256 MMAs per K step that share the
 // A stage, so a CTA pulls 25% fewer operand bytes from L2 per MMA.  Both halves
 // fill all 512 TMEM columns, so there is a single accumulator: the next unit's
 // MMAs wait for the epilogue (worth it where units are long, as in dH).
-// XF = 1 (2-CTA pairs, bf16, store / accumulate epilogues): the A operand is a
-// stage of stored exponentials that the transform warps turn into dS.  Each
-// CTA's copies then complete on its own barriers (the transform warps of both
-// CTAs wait for them), and the MMA issuer waits for the transforms of both
-// CTAs on a third ring of barriers.
+// XF = 1 (dH: 2-CTA pairs, bf16, K-major A, store / accumulate epilogues): the
+// A operand is a stage of stored exponentials that the transform warps turn
+// into dS.  Each CTA's copies then complete on its own barriers (the transform
+// warps of both CTAs wait for them), the MMA issuer waits for the transforms
+// of both CTAs on a third ring of barriers, and a stage is refilled only after
+// the MMAs and the transform warps' dS stores (tmD) have read it.
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
 __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
-  static_assert(!XF || (PAIR && sizeof(Elem) == 2 && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
-                "operand transform: bf16 2-CTA pairs with a store or accumulate epilogue");
+  static_assert(!XF || (PAIR && sizeof(Elem) == 2 && A_MN == 0 &&
+                        (EPI == EPI_STORE || EPI == EPI_ACCUM)),
+                "operand transform: bf16 2-CTA pairs, K-major A, store or accumulate");
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
@@ -298,11 +300,6 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       idesc_dense(ElemTraits<Elem>::kFmt, kBM * kCtas, kBN, A_MN, B_MN);
   // copies of each CTA complete on its own barriers (else on the leader's)
   constexpr bool kLocalCopies = XF || !PAIR;
-  // dW with the operand transform: the stage's token scales ride with the stage,
-  // in slots at the end of the barrier region
-  constexpr bool kXfW = XF && A_MN;
-  constexpr int kXfSlotOffset = 512;  // barriers and flags use less
-  static_assert(!kXfW || kXfSlotOffset + kNS * kXfScaleBytes <= kBarrierRegion, "scale slots");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -317,8 +314,6 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* issued_slot = tmem_slot + 2;  // stages whose copies this CTA's producer issued
-  float* xf_slot = reinterpret_cast<float*>(smem + kRingBytes + kXfSlotOffset);  // [kNS][64]
-  static_assert(3 * kStagesPair * 8 + 5 * 8 + 3 * 4 <= kXfSlotOffset, "barrier region");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -331,8 +326,8 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-      mbar_init(&ready_bar[s], kCtas);  // one arrival per CTA (the stage's transform warp)
+      mbar_init(&empty_bar[s], XF ? 1 + 4 : 1);  // MMA commit (+ each transform warp)
+      mbar_init(&ready_bar[s], 4 * kCtas);        // one arrival per transform warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -385,14 +380,10 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
           }
           uint8_t* a_s = smem + s * kSBytes;
           uint8_t* b_s = a_s + kATileBytes;
-          if (kLocalCopies) mbar_arrive_expect_tx(&full_bar[s], kSBytes + (kXfW ? kXfScaleBytes : 0));
+          if (kLocalCopies) mbar_arrive_expect_tx(&full_bar[s], kSBytes);
           else if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
           const uint32_t fb = kLocalCopies ? 0u : mapa_shared(&full_bar[s], 0);
           const int k0 = kb * kBKe;
-          if (kXfW)  // the stage's 64 token scales of this CTA's vocabulary tile
-            bulk_load_1d(xf_slot + s * (kXfScaleBytes / 4),
-                         p.xf_sc + static_cast<int64_t>(m0 >> 8) * p.xf_ld + k0, kXfScaleBytes,
-                         &full_bar[s]);
 #pragma unroll
           for (int sl = 0; sl < (A_MN ? kBM / kMNe : 1); ++sl) {
             void* dst = a_s + sl * kSlabBytes;
@@ -488,60 +479,77 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     __syncwarp();
   } else if (XF && warp >= 6) {
     // ------------------------------------------------------------ operand transform
-    // Transform warp xw scales this CTA's A stages n = xw, xw + 4, ... (four
-    // stages in flight), each lane four of the stage's 128 rows of 128 bytes:
-    //   dH (A = dS [rows][V], K-major): logit rows m0 + lane + 32 i, with the
-    //      stage's tile scales loaded before the stage's data is waited for;
-    //   dW (A = dS^T, slabs [64 tokens][64 columns]): token rows of the slabs,
-    //      scales from the slot the producer filled with the stage.
+    // Warp xw of the four scales rows 32 xw .. 32 xw + 31 of this CTA's A stage
+    // (logit rows m0 + xt), lane = row, with the row's scale for the stage's
+    // 256-column tile kept in a register and loaded one tile (4 stages) ahead.
     // The rows written are read only by this CTA's tensor core (each CTA of a
     // pair supplies its own 128 rows of A), so the proxy fence and a CTA-scope
-    // release on the arrival order them before the leader issues the MMAs.
+    // arrival order them before the leader issues the MMAs.  With p.xf_store,
+    // the unit of output column tile xw mod tiles_n also stores the warp's 32
+    // formed rows to the dS chunk (so every row is stored once and the stores
+    // spread over the column tiles); a stored stage is released for refilling
+    // one stage later, once its store has read it.
     const int xw = warp - 6;
+    const int xt = xw * 32 + lane;  // 0 .. 127
     uint32_t n = 0;
     bool ok = true;
+    int pend = -1;  // stage whose store may still be reading it (lane 0)
+    // the dS chunk is read back only by the next kernel: keep it from evicting
+    // the e and W tiles that this kernel's other column tiles re-read from L2
+    const uint64_t ds_policy = l2_policy_evict_first();
     for (int t = unit; t < total_tiles && ok; t += units) {
       const UnitRange ur = unit_range(t, p);
       int tm, tn;
       tile_coords(ur.tile, p, tm, tn);
       const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;
+      const int row = m0 + xt;
+      const bool live = row < p.xf_rows;
+      const bool store =
+          p.xf_store != 0 && tn == xw % p.tiles_n && m0 + xw * 32 < p.xf_rows;
+      int cur_t = -1, nxt_t = -1;
+      float cur = 0.f, nxt = 0.f;
       for (int kb = ur.kb0; kb < ur.kb1; ++kb, ++n) {
-        if (static_cast<int>(n & 3u) != xw) continue;
         const uint32_t s = n % kNS;
         const uint32_t ph = (n / kNS) & 1u;
         const int k0 = kb * kBKe;
-        float sc[4];
-        if (A_MN == 0) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = m0 + lane + 32 * i;
-            sc[i] = row < p.xf_rows
-                        ? __ldg(p.xf_sc + static_cast<int64_t>(k0 >> 8) * p.xf_ld + row)
-                        : 0.f;
-          }
+        if (live && (k0 >> 8) != cur_t) {  // entering a new 256-column tile
+          cur_t = k0 >> 8;
+          cur = (nxt_t == cur_t) ? nxt : __ldg(p.xf_sc + static_cast<int64_t>(cur_t) * p.xf_ld + row);
+          nxt_t = cur_t + 1;
+          if (nxt_t * 256 < p.num_kb * kBKe)  // prefetch the next tile's scale
+            nxt = __ldg(p.xf_sc + static_cast<int64_t>(nxt_t) * p.xf_ld + row);
         }
         if (!wait_bar(&full_bar[s], ph, ctl, true)) {
           ok = false;
           break;
         }
-        uint8_t* a_s = smem + s * kSBytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = lane + 32 * i;  // 0 .. 127
-          if (A_MN == 0) {
-            if (m0 + r < p.xf_rows)
-              xf_row(a_s + r * kRowBytes, r & 7, __float2bfloat162_rn(sc[i]));
-          } else {
-            const int kk = r & 63;
-            if (k0 + kk < p.xf_rows)
-              xf_row(a_s + (r >> 6) * kSlabBytes + kk * kRowBytes, kk & 7,
-                     __float2bfloat162_rn(xf_slot[s * (kXfScaleBytes / 4) + kk]));
-          }
-        }
-        fence_proxy_async_smem();  // generic writes -> the tensor core's reads
+        uint8_t* rows = smem + s * kSBytes + xw * 32 * kRowBytes;  // this warp's 4 KB
+        if (live) xf_row(rows + lane * kRowBytes, lane & 7, __float2bfloat162_rn(cur));
+        fence_proxy_async_smem();  // generic writes -> the tensor core's and TMA's reads
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(&ready_bar[s], 0));
+        if (lane == 0) {
+          if (store) {
+            tma_store_2d_hint(&tmD, rows, k0, m0 + xw * 32, ds_policy);
+            bulk_commit();
+          }
+          mbar_arrive_cluster(mapa_shared(&ready_bar[s], 0));
+          if (pend >= 0) {  // the previous stored stage: its store has read it
+            if (store) bulk_wait_read_1();
+            else bulk_wait_read_0();
+            mbar_arrive(&empty_bar[pend]);
+            pend = -1;
+          }
+          if (store) pend = static_cast<int>(s);
+          else mbar_arrive(&empty_bar[s]);
+        }
       }
+    }
+    if (lane == 0) {
+      if (ok && pend >= 0) {
+        bulk_wait_read_0();
+        mbar_arrive(&empty_bar[pend]);
+      }
+      bulk_wait_all();  // the dS stores have landed before exit
     }
     __syncwarp();
   } else if (warp < 4) {

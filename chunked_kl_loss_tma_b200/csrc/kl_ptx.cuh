@@ -76,17 +76,6 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
-// Contiguous (untiled) bulk copy of `bytes` from global to this CTA's shared
-// memory, completion counted on bar (16-byte aligned addresses and size).
-__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
-                                             uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // 2-D tiled load issued by either CTA of a 2-CTA pair; the transaction bytes
 // are counted on the barrier at shared::cluster address bar_cluster (the
 // leader CTA's barrier).
@@ -145,6 +134,10 @@ __device__ __forceinline__ void bulk_commit() {
 // Wait until at most one committed bulk group still reads shared memory.
 __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// Wait until no committed bulk group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // Wait until every committed bulk group has completed.
 __device__ __forceinline__ void bulk_wait_all() {
