@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--entry", default="fused", choices=["fused", "split"],
                     help="fused: kl_fwd_bwd; split: kl_fwd then kl_bwd (the autograd path, "
                          "backward recomputes the logits)")
+    ap.add_argument("--recompute-all", action="store_true",
+                    help="--entry split: the backward recomputes every chunk (by default, as "
+                         "the autograd path, kl_fwd keeps the last chunk's logits for kl_bwd)")
     ap.add_argument("--parallel", default="tokens", choices=["tokens", "vocab"],
                     help="tokens: each rank its own token shard, no collective (weak scaling); "
                          "vocab: the head split by vocabulary rows over the ranks, the same "
@@ -257,6 +260,7 @@ def gpu_arm(args):
         comm = vpm.TorchComm()
 
     if args.entry == "split":
+        prob.keep_last_chunk = 0 if args.recompute_all else 1
         ws_split = max(ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD),
                        ops.workspace_bytes(prob, _lib.KL_ENTRY_BWD))
         if ws_split > ws_bytes:
@@ -359,9 +363,21 @@ def gpu_arm(args):
             for i in range(n):
                 stager.acquire(slot, cstream)
                 nxt = stager.put(host) if i + 1 < n else None
-                _lib.check(_lib.kl_fwd_bwd(probs[slot][0], workspace.data_ptr(), ws_bytes, 1.0,
-                                           loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(),
-                                           0, stream), "kl_fwd_bwd")
+                pr = probs[slot][0]
+                if args.entry == "split":
+                    pr.keep_last_chunk = prob.keep_last_chunk
+                    _lib.check(_lib.kl_fwd(pr, workspace.data_ptr(), ws_bytes, loss.data_ptr(),
+                                           lse_s.data_ptr(),
+                                           None if lse_t is None else lse_t.data_ptr(), None,
+                                           stream), "kl_fwd")
+                    _lib.check(_lib.kl_bwd(pr, workspace.data_ptr(), ws_bytes, lse_s.data_ptr(),
+                                           None if lse_t is None else lse_t.data_ptr(),
+                                           g_one.data_ptr(), dH.data_ptr(), dW.data_ptr(), 0,
+                                           stream), "kl_bwd")
+                else:
+                    _lib.check(_lib.kl_fwd_bwd(pr, workspace.data_ptr(), ws_bytes, 1.0,
+                                               loss.data_ptr(), None, dH.data_ptr(),
+                                               dW.data_ptr(), 0, stream), "kl_fwd_bwd")
                 stager.release(slot, cstream)
                 if dp_sync != "none":
                     dp_reduce()
@@ -473,8 +489,12 @@ def gpu_arm(args):
         line["config"]["N"] = N
     if args.entry == "split":
         line["metric"] += " [kl_fwd + kl_bwd]"
-        # backward recomputes the student (and teacher) logits once more
-        executed = step_flops + 2.0 * N * V * (d + (w.d_t if w.mode == "hidden" else 0))
+        line["config"]["keep_last_chunk"] = not args.recompute_all
+        # backward recomputes the student (and teacher) logits of every chunk
+        # (but the last one, when kept)
+        C = args.chunk or 4096
+        n_re = N if args.recompute_all else max(N - (N - 1) % C - 1, 0) if N > C else 0
+        executed = step_flops + 2.0 * n_re * V * (d + (w.d_t if w.mode == "hidden" else 0))
         line["executed_tflops_step"] = round(executed * args.steps / (ms / 1e3) / 1e12, 1)
     print(json.dumps(line), flush=True)
 

@@ -6,19 +6,16 @@
 // KL": the output projection is fused into the loss, each logit chunk is
 // transient, and backward recomputes one projection per chunk).
 //
-// Per chunk of C token rows (fwd_bwd, top-K, bf16):
+// Per chunk of C token rows (fwd_bwd, top-K):
 //   prep_topk      cache -> sorted ids + teacher probabilities q, m, sum q log q
 //   gemm STATS     S~ = H_c W^T / T  (tcgen05), split-V row statistics + gather,
-//                  stores e = 2^(s~ log2 e - tile max)
+//                  stores s~ - tile max
 //   row_reduce     lse_s, row loss
-//   xf_patch       -c q folded into e at the cached columns
-//   xf_scales      per (tile, row) scale with dS = scale * e
-//   gemm ACCUM     dH_c = dS W: wide 256 x 512 tiles, split-K fp32 parts, dS
-//                  formed from e in shared memory by the transform warps
+//   dlogits_topk   S~ -> dS in place
+//   gemm ACCUM     dH_c = dS W: wide 256 x 512 tiles, split-K fp32 parts
 //   splitk_reduce  the parts summed in a fixed order -> dH_c
-//   gemm ACCUM     dW (+)= dS^T H_c, dS formed the same way
-// then finalize_loss (masked mean).  No host synchronisation anywhere.  fp32
-// inputs store s~ - tile max and turn it into dS with the dlogits_topk pass.
+//   gemm ACCUM     dW (+)= dS^T H_c
+// then finalize_loss (masked mean).  No host synchronisation anywhere.
 // The teacher-hidden mode runs the teacher pass (fp32 t~ - tile max) and then
 // the student pass, whose epilogue forms the per-tile loss sums against the
 // teacher tile; hidden_sums merges them into lse_s, lse_t, the row loss and
@@ -210,13 +207,6 @@ struct Plan {
   // current chunk of H or Ht) and K-major copies W^T [d][Vp], dS^T [V][Cp],
   // H_c^T [d][Cp] for the gradient contractions.
   int64_t Cp = 0;
-  // bf16 top-K: the logits pass stores exponentials and the gradient
-  // contractions form dS from them as their operand stages arrive (no dlogits
-  // pass); fp32 keeps the dlogits pass (its operands are transposed copies)
-  bool xf = false;
-  int64_t Cx = 0;          // (xf) row stride of the transposed dS scales: C rounded up to 64
-  size_t off_xsc = 0;      // (xf) dS scales [tiles_v][Cx] fp32
-  size_t off_dsbuf = 0;    // (xf) dS chunk [C][Vp] bf16
   size_t off_ubar = 0;     // (hidden) u_bar per chunk row
   int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
   size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
@@ -267,6 +257,7 @@ int validate_shape(const kl_problem* p) {
   if (!(p->reverse_weight >= 0.f && p->reverse_weight <= 1.f) ||
       (p->reverse_weight > 0.f && p->teacher != KL_TEACHER_HIDDEN))
     return KL_ERR_ARG;
+  if (p->keep_last_chunk != 0 && p->keep_last_chunk != 1) return KL_ERR_ARG;
   if (p->v_begin < 0 || p->V_total < 0 || p->V_total > (int64_t(1) << 31) - 512 ||
       (p->V_total > 0 && p->v_begin + p->V > p->V_total) || (p->V_total == 0 && p->v_begin != 0))
     return KL_ERR_ARG;
@@ -303,6 +294,8 @@ int64_t vocab_total(const kl_problem* p) { return p->V_total > 0 ? p->V_total : 
 bool whole_head(const kl_problem* p) { return p->v_begin == 0 && vocab_total(p) == p->V; }
 
 Plan make_plan(const kl_problem* p, int entry) {
+  // a kept chunk passes from kl_fwd to kl_bwd in one layout: the fused pass's
+  if (p->keep_last_chunk) entry = KL_ENTRY_FWD_BWD;
   Plan pl;
   pl.eb = p->dtype == KL_DTYPE_BF16 ? 2 : 4;
   pl.hidden = p->teacher == KL_TEACHER_HIDDEN;
@@ -311,7 +304,6 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (pl.C < 1) pl.C = 1;
   pl.Vp = cdiv(p->V, 8) * 8;
   pl.tiles_v = static_cast<int>(cdiv(p->V, kBN));
-  pl.xf = pl.eb == 2 && !pl.hidden;
   // student logits / dS chunk: wherever dS is formed (not the forward alone)
   const bool need_sbuf = entry != KL_ENTRY_FWD;
   // tile statistics: every pass that computes them (the top-K backward forms
@@ -331,11 +323,6 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (need_stats && pl.hidden)
     pl.off_pt = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
   if (pl.hidden && entry != KL_ENTRY_FWD) pl.off_ubar = take(static_cast<size_t>(pl.C) * 4);
-  if (pl.xf && entry == KL_ENTRY_FWD_BWD) {
-    pl.Cx = cdiv(pl.C, 64) * 64;
-    pl.off_xsc = take(static_cast<size_t>(pl.tiles_v) * pl.Cx * 4);
-    pl.off_dsbuf = take(buf);  // dS chunk, formed by the dH contraction for dW
-  }
   if (!pl.hidden) {
     pl.off_sidx = take(static_cast<size_t>(pl.C) * p->K * 4);
     pl.off_sq = take(static_cast<size_t>(pl.C) * p->K * 4);
@@ -371,11 +358,10 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
-                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops,
-                const CUtensorMap* md = nullptr) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
+                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -391,7 +377,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(XF ? kGemmThreadsXf : kGemmThreads);
+  cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = st;
   if (PAIR) {
@@ -405,7 +391,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md != nullptr ? *md : mc, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, gp);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
@@ -449,13 +435,13 @@ int prepare_heads(Ctx& c) {
 }
 
 // Logits pass over one chunk: S~ = X_c . Wh^T / T with the tile statistics in
-// `partials`.  store: STORE_NONE, STORE_SHIFTED (s~ - tile max into `out`, fp32
-// when out_f32, else the input type) or STORE_EXP (bf16 exponentials).  tbuf /
-// tpart: the teacher pass's stored tile and statistics (student pass of the
-// teacher-hidden mode: the tile sums A and U go to partials .z / .w).
+// `partials`; out != nullptr: s~ - tile max stored into `out` (fp32 when
+// out_f32, else the input type).  tbuf / tpart: the teacher pass's stored tile
+// and statistics (student pass of the teacher-hidden mode: the tile sums A and
+// U go to partials .z / .w).
 template <typename Elem>
 int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, int64_t Cn,
-                void* out, int store, bool out_f32, float4* partials, const int* sidx,
+                void* out, bool out_f32, float4* partials, const int* sidx,
                 const float* sq, int ktop, const char* name, const float* tbuf = nullptr,
                 const float4* tpart = nullptr) {
   const kl_problem* p = c.p;
@@ -471,10 +457,9 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   if (!make_map(&ma, xc, p->dtype, dx, Cn, dx * sizeof(Elem), kBKe, kBM) ||
       !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2))
     return KL_ERR_CUDA;
-  if (store != STORE_NONE) {
-    const bool f32 = out_f32 && store == STORE_SHIFTED;
-    if (!make_out_map(&mc, out, f32 ? KL_DTYPE_F32 : p->dtype, p->V, Cn,
-                      c.pl.Vp * (f32 ? 4 : sizeof(Elem))))
+  if (out != nullptr) {
+    if (!make_out_map(&mc, out, out_f32 ? KL_DTYPE_F32 : p->dtype, p->V, Cn,
+                      c.pl.Vp * (out_f32 ? 4 : sizeof(Elem))))
       return KL_ERR_CUDA;
   } else {
     mc = mb;  // statistics only: the output map is not used
@@ -484,7 +469,7 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.tiles_n = c.pl.tiles_v;
   gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
   gp.m_fastest = 1;
-  gp.store = store;
+  gp.store = out != nullptr;
   gp.out_f32 = out_f32 ? 1 : 0;
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
@@ -609,28 +594,17 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
 
 // dH_c = dS . W and dW (+)= dS^T . H_c for chunk rows [c0, c0 + Cn) from the
 // chunk buffer dS.  dH_f32: write dH as fp32 (a vocabulary shard's partial sum)
-// whatever Elem is.  XF = 1: the buffer holds the logits pass's exponentials,
-// patched at the cached columns (xf_patch_kernel); the dH contraction forms
-// dS = scale * e in shared memory with the per-(tile, row) scales xf_sc and
-// stores it to the workspace's dS chunk, which the dW contraction reads.
-template <typename Elem, int XF>
-int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
-                    bool dH_f32, const float* xf_sc) {
+// whatever Elem is.
+template <typename Elem>
+int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+               bool dH_f32 = false) {
+  if (sizeof(Elem) == 4)
+    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   constexpr int kMNe = kRowBytes / sizeof(Elem);
   const int64_t d = p->d;
   const uint64_t ldS = c.pl.Vp * sizeof(Elem);
-  Elem* dS_formed = XF ? reinterpret_cast<Elem*>(c.ws + c.pl.off_dsbuf) : dS;
-  CUtensorMap md;  // XF: the dS chunk written by the dH contraction, 64 x 32 boxes
-  if (XF && !make_map(&md, dS_formed, p->dtype, p->V, Cn, ldS, kBKe, 32)) return KL_ERR_CUDA;
-  auto set_xf = [&](GemmParams& gp) {
-    if (!XF) return;
-    gp.xf_sc = xf_sc;
-    gp.xf_ld = c.pl.Cx;
-    gp.xf_rows = static_cast<int>(Cn);
-    gp.xf_store = 1;
-  };
   // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.  When the
   // output has too few tiles to fill the GPU, V is split into ksplit parts whose
   // fp32 partial products are summed in a fixed order afterwards.
@@ -648,7 +622,6 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
-    set_xf(gp);
     int ks = choose_ksplit(static_cast<int64_t>(gp.tiles_m) * gp.tiles_n, gp.num_kb, c.sms / 2);
     if (ks > c.pl.ksplit_dh) ks = c.pl.ksplit_dh;
     if (ks > 1) {
@@ -663,9 +636,8 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
       CUtensorMap mc;
       if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d,
-                                                                 XF ? &md : nullptr)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
+                                                             gp, 2.0 * Cn * p->V * d)));
       LaunchScope ls("splitk_reduce", c.st, 0,
                      (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
       if (dH_f32)
@@ -681,24 +653,22 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d,
-                                                                 XF ? &md : nullptr)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
+                                                             gp, 2.0 * Cn * p->V * d)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
                         d * sizeof(Elem)))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
-                                                                 mc, gp, 2.0 * Cn * p->V * d,
-                                                                 XF ? &md : nullptr)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
+                                                             gp, 2.0 * Cn * p->V * d)));
     }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
   {
     CUtensorMap ma, mb, mc;
     const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * d * sizeof(Elem);
-    if (!make_map(&ma, dS_formed, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
+    if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
         !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe) ||
         !make_out_map(&mc, dW, KL_DTYPE_F32, d, p->V, d * 4))
       return KL_ERR_CUDA;
@@ -716,19 +686,6 @@ int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* d
                                                   2.0 * Cn * p->V * d)));
   }
   return KL_OK;
-}
-
-// dH_f32: write dH as fp32 (a vocabulary shard's partial sum) whatever Elem is.
-// xf_sc != nullptr: dS is formed in the contractions' operand path (bf16).
-template <typename Elem>
-int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
-               bool dH_f32 = false, const float* xf_sc = nullptr) {
-  if (sizeof(Elem) == 4)
-    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
-  using B = __nv_bfloat16;
-  B* b = reinterpret_cast<B*>(dS);
-  return xf_sc != nullptr ? gemm_grads_bf16<B, 1>(c, b, c0, Cn, dH, dW, beta, dH_f32, xf_sc)
-                          : gemm_grads_bf16<B, 0>(c, b, c0, Cn, dH, dW, beta, dH_f32, nullptr);
 }
 
 int launch_count_valid(Ctx& c) {
@@ -831,35 +788,6 @@ int launch_dlogits_full(Ctx& c, Elem* S, const float* Tt, int64_t c0, int64_t Cn
   return KL_LAUNCHED();
 }
 
-// dS from the stored exponentials of chunk rows [c0, c0 + Cn) (top-K, bf16):
-// the cached columns' corrections folded into the buffer S, then the
-// transposed per-(tile, row) scales.  lse: the whole problem's rows.  Returns
-// the scales for gemm_grads.
-int launch_xf_prep(Ctx& c, __nv_bfloat16* S, int64_t c0, int64_t Cn, const float* lse,
-                   const float* g_dev, float g_host, const float** xf_sc) {
-  const kl_problem* p = c.p;
-  const float4* part = reinterpret_cast<const float4*>(c.ws + c.pl.off_ps);
-  const float2* rinfo = reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo);
-  const uint8_t* mask = p->mask ? p->mask + c0 : nullptr;
-  const float* T_row = p->T_row ? p->T_row + c0 : nullptr;
-  float* sc_out = reinterpret_cast<float*>(c.ws + c.pl.off_xsc);
-  {
-    LaunchScope ls("xf_patch", c.st, 0, static_cast<double>(Cn) * p->K * 16);
-    xf_patch_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
-        S, c.pl.Vp, part, c.pl.tiles_v, static_cast<int>(Cn), static_cast<int>(p->V), lse + c0,
-        mask, rinfo, reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
-        reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT,
-        T_row);
-    KL_TRY(KL_LAUNCHED());
-  }
-  LaunchScope ls("xf_scales", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 20);
-  xf_scales_kernel<<<static_cast<unsigned>(cdiv(Cn, 32)), 256, 0, c.st>>>(
-      part, c.pl.tiles_v, static_cast<int>(Cn), lse + c0, mask, rinfo, c.sc, g_dev, g_host,
-      c.invT, T_row, sc_out, c.pl.Cx);
-  *xf_sc = sc_out;
-  return KL_LAUNCHED();
-}
-
 // Teacher-hidden row sums of chunk rows [c0, c0 + Cn) (hidden_sums_kernel).
 // lse_*_in: given log-sum-exps (whole arrays, or nullptr to merge them from the
 // tile statistics into lse_*_out); the other outputs as the kernel's, each
@@ -890,11 +818,10 @@ int hidden_logits(Ctx& c, int64_t c0, int64_t Cn, bool store_student) {
   float* Tt = reinterpret_cast<float*>(c.ws + c.pl.off_tbuf);
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
   float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
-  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, STORE_SHIFTED, true, pt,
+  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, true, pt,
                            nullptr, nullptr, 0, "gemm_teacher_logits"));
   return gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn,
-                           store_student ? c.ws + c.pl.off_sbuf : nullptr,
-                           store_student ? STORE_SHIFTED : STORE_NONE, sizeof(Elem) == 4, ps,
+                           store_student ? c.ws + c.pl.off_sbuf : nullptr, sizeof(Elem) == 4, ps,
                            nullptr, nullptr, 0, "gemm_logits_stats", Tt, pt);
 }
 
@@ -940,15 +867,18 @@ int run_fwd(Ctx& c, float* loss, float* lse_s, float* lse_t, float* row_loss) {
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
   for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
     const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
+    // keep_last_chunk: the last chunk's logits stay in the student buffer
+    const bool keep = p->keep_last_chunk && c0 + Cn == p->N;
     if (!c.pl.hidden) {
       KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, nullptr, STORE_NONE, false, ps,
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn,
+                               keep ? c.ws + c.pl.off_sbuf : nullptr, sizeof(Elem) == 4, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                                "gemm_logits_stats"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
     } else {
-      KL_TRY(hidden_logits<Elem>(c, c0, Cn, false));
+      KL_TRY(hidden_logits<Elem>(c, c0, Cn, keep));
       KL_TRY(launch_hidden_sums(c, c0, Cn, nullptr, nullptr, lse_s, lse_t, 1, rl, nullptr,
                                 nullptr));
     }
@@ -967,21 +897,31 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
   if (sizeof(Elem) == 4)
     KL_TRY(launch_transpose(c, static_cast<const float*>(p->W), p->d,
                             reinterpret_cast<float*>(c.ws + c.pl.off_wT), c.pl.Vp, p->V, p->d));
-  for (int64_t c0 = 0; c0 < p->N; c0 += c.pl.C) {
+  const int64_t nch = cdiv(p->N, c.pl.C);
+  // keep_last_chunk: the last chunk first, from the logits kl_fwd left behind
+  for (int64_t i = 0; i < nch; ++i) {
+    const int64_t k = p->keep_last_chunk ? (i == 0 ? nch - 1 : i - 1) : i;
+    const bool kept = p->keep_last_chunk && i == 0;
+    const int64_t c0 = k * c.pl.C;
     const int64_t Cn = (p->N - c0) < c.pl.C ? (p->N - c0) : c.pl.C;
     if (!c.pl.hidden) {
-      KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_dlogits<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
+      if (kept) {  // s~ - tile max, the tile statistics and the prepared cache are in ws
+        KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host,
+                                         reinterpret_cast<const float4*>(c.ws + c.pl.off_ps)));
+      } else {
+        KL_TRY(launch_prep(c, c0, Cn));
+        KL_TRY(gemm_dlogits<Elem>(c, S, c0, Cn, lse_s, g_dev, g_host));
+      }
     } else {
-      // both logits recomputed; u_bar from the given lse's
+      // both logits recomputed (or kept); u_bar from the given lse's
       float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
-      KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
+      if (!kept) KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
       KL_TRY(launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, 1, nullptr, nullptr,
                                 ubar));
       KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
                                        c0, Cn, lse_s, lse_t, ubar, g_dev, g_host));
     }
-    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || c0 > 0) ? 1 : 0));
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || i > 0) ? 1 : 0));
   }
   return KL_OK;
 }
@@ -1009,19 +949,11 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
     const int beta = (accumulate || c0 > 0) ? 1 : 0;
     if (!c.pl.hidden) {
       KL_TRY(launch_prep(c, c0, Cn));
-      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S,
-                               c.pl.xf ? STORE_EXP : STORE_SHIFTED, sizeof(Elem) == 4, ps,
+      KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                                "gemm_logits_stats"));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
-      if (c.pl.xf) {
-        const float* xsc = nullptr;
-        KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
-                              &xsc));
-        KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, false, xsc));
-        continue;
-      }
       KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
     } else {
       float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
@@ -1061,8 +993,7 @@ int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
   float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
   if (!c.pl.hidden) {
     KL_TRY(launch_prep(c, c0, Cn));
-    KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S,
-                             c.pl.xf ? STORE_EXP : STORE_SHIFTED, sizeof(Elem) == 4, ps,
+    KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                              reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                              reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
                              "gemm_logits_stats"));
@@ -1121,15 +1052,8 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sum
   const int beta = (accumulate || k > 0) ? 1 : 0;
   KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, lse_user, rl));
   if (!c.pl.hidden) {
-    if (c.pl.xf) {
-      const float* xsc = nullptr;
-      KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
-                            &xsc));
-      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true, xsc));
-    } else {
-      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
-      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
-    }
+    KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
+    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
   } else {
     // this shard's A, U (its row-loss share) and u_bar, the sum of every shard's
     // U when the reverse KL needs it (its sums came through the second exchange)
@@ -1149,6 +1073,7 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sum
 int vp_begin(const kl_problem* p, int64_t chunk, void* ws, size_t ws_bytes, void* stream,
              Ctx& c) {
   KL_TRY(validate(p));
+  if (p->keep_last_chunk) return KL_ERR_ARG;
   if (chunk < 0 || chunk >= num_chunks(p, make_plan(p, KL_ENTRY_FWD_BWD).C)) return KL_ERR_ARG;
   return begin(p, KL_ENTRY_FWD_BWD, ws, ws_bytes, stream, c, true);
 }
@@ -1192,6 +1117,7 @@ int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,
 
 int kl_fwd_bwd(const kl_problem* p, void* ws, size_t ws_bytes, float grad_loss, float* loss,
                float* row_loss, void* dH, float* dW, int accumulate_dW, void* stream) {
+  if (p != nullptr && p->keep_last_chunk) return KL_ERR_ARG;
   Ctx c;
   KL_TRY(begin(p, KL_ENTRY_FWD_BWD, ws, ws_bytes, stream, c));
   if (loss == nullptr || dW == nullptr || (p->N > 0 && dH == nullptr)) return KL_ERR_NULL;
@@ -1359,6 +1285,7 @@ int noalloc_scratch(uint8_t** out) {
 
 extern "C" int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
                               int* status, void* stream) {
+  if (p != nullptr && p->keep_last_chunk) return KL_ERR_ARG;
   KL_TRY(validate(p));
   if (!whole_head(p)) return KL_ERR_ARG;
   if (p->dtype != KL_DTYPE_BF16 || p->teacher != KL_TEACHER_TOPK) return KL_ERR_DTYPE;

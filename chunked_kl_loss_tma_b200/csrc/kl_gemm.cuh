@@ -1,9 +1,8 @@
 // kl_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for the three
 // contractions of the fused KL loss, with the loss arithmetic fused into the
-// epilogue and, for the gradient contractions, into the operand path
-// ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and a
-// Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection is
-// integrated into the loss and each logit chunk is transient).
+// epilogue ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits
+// and a Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection
+// is integrated into the loss and each logit chunk is transient).
 //
 //   C[M, N] = A[M, K] . B[N, K]^T   (bf16 -> kind::f16, fp32 -> kind::tf32;
 //                                     fp32 accumulation in TMEM)
@@ -12,9 +11,7 @@
 //              max and sum of 2^(s~ log2 e - max) and the cross term
 //              sum_i q_i s~_{idx_i} of the cached top-K entries that fall in
 //              the tile (gathered from the fp32 accumulator).  Optionally
-//              stores s~ - max (store = 1; natural units) or the exponentials
-//              2^(s~ log2 e - max) themselves (store = 2), which the gradient
-//              contractions scale into dS as their operand stages arrive.  In
+//              stores s~ - max (natural units; fp32 or the input type).  In
 //              the teacher-hidden mode the student pass also reads the
 //              teacher tile (stored fp32 by the teacher pass) and forms the
 //              tile's sums sum p_t (t~ - s~) and sum p_s (s~ - t~) from fp32.
@@ -38,14 +35,7 @@
 //   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
-//   warp 5     TMEM allocator + MMA issuer (one thread);
-//   warps 6-9  (XF = 1 only, dH) operand transform: turn the A stage -- the
-//              stored exponentials e = 2^(s~ log2 e - tile max) of a logit
-//              chunk, already corrected at the cached entries -- into
-//              dS = scale(row, tile) * e in shared memory before the MMAs read
-//              it, and (units of output column tile 0) store the formed stage
-//              as the dS chunk that the dW contraction then reads.  This is
-//              the dlogits step of the loss without its own pass over HBM.
+//   warp 5     TMEM allocator + MMA issuer (one thread).
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
 // the 512 columns with one 256 x 512 tile (see the template below).  In the
@@ -74,7 +64,6 @@ constexpr int kATileBytes = kBM * kRowBytes;
 constexpr int kBTileBytes = kBN * kRowBytes;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
-constexpr int kGemmThreadsXf = 320;  // + four operand-transform warps
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kRingBytes = kStages * kStageBytes;          // 192 KB operand ring
 constexpr int kBarrierRegion = 1024;                        // barriers, TMEM slot, flags
@@ -94,36 +83,26 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2f = 0.6931471805599453f;
 
 enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3 };
-// EPI_STATS store modes
-enum { STORE_NONE = 0, STORE_SHIFTED = 1, STORE_EXP = 2 };
 
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
-  int store;           // STATS: STORE_NONE / STORE_SHIFTED / STORE_EXP
-  int out_f32;         // STATS, STORE_SHIFTED: the output map holds fp32
+  int store;           // STATS: store s~ - tile max through the output map (0 = statistics only)
+  int out_f32;         // STATS with store: the output map holds fp32
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
   float scale;         // STATS / DLOGITS: 1 / T
   const float* T_row;  // STATS / DLOGITS: per-row temperature (chunk rows), or nullptr
   int beta;            // ACCUM: 0 overwrite, 1 accumulate
-  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross | A, gather start | U)
-  const int* sidx;     // STATS gather / XF corrections: [rows][ktop] ascending ids,
-                       // INT_MAX = empty
-  const float* sq;     // STATS gather / XF corrections: [rows][ktop] teacher probabilities
+  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross | A, 0 | U)
+  const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
+  const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
   // STATS, student pass of the teacher-hidden mode: the teacher tile stored by
   // the teacher pass (t~ - tile max, fp32, row stride tld) and its statistics
   const float* tbuf;
   int64_t tld;
   const float4* tpart;
-  // XF: scale of dS per (256-column tile, logit row), [tiles][xf_ld] fp32
-  // (xf_ld a multiple of 64), so that dS = scale * e for the stored e
-  const float* xf_sc;
-  int64_t xf_ld;
-  int xf_rows;         // logit rows (tokens) that exist
-  int xf_store;        // XF: the units of output column tile 0 store each formed
-                       // dS stage through the fourth map (the dS chunk for dW)
   // DLOGITS: per-row lse (natural units), (m, .) per row, mask, and the scalars
   // of c = g / (n T): the loss normaliser n, and g (device pointer or value)
   const float* lse;
@@ -235,46 +214,18 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// XF: one 128-byte row of a dS operand stage (64 bf16 values of one logit row
-// within one 256-column tile), x -> x * scale in place with packed bf16x2
-// multiplies (scale rounded to bf16: with the product's rounding, 2^-8
-// relative error per entry).  The chunks are visited in the row's swizzled
-// order (chunk j at position j ^ sw) so that the 32 rows a warp's lanes touch
-// at once hit all 32 banks.
-__device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 scale2) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    uint4* cp = reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4));
-    uint4 u = *cp;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], scale2);
-    *cp = u;
-  }
-}
-
 // WIDE = 1 (2-CTA pairs, store / accumulate epilogues): each work unit is a
 // 256 x 512 output tile computed as two N = 256 MMAs per K step that share the
 // A stage, so a CTA pulls 25% fewer operand bytes from L2 per MMA.  Both halves
 // fill all 512 TMEM columns, so there is a single accumulator: the next unit's
 // MMAs wait for the epilogue (worth it where units are long, as in dH).
-// XF = 1 (dH: 2-CTA pairs, bf16, K-major A, store / accumulate epilogues): the
-// A operand is a stage of stored exponentials that the transform warps turn
-// into dS.  Each CTA's copies then complete on its own barriers (the transform
-// warps of both CTAs wait for them), the MMA issuer waits for the transforms
-// of both CTAs on a third ring of barriers, and a stage is refilled only after
-// the MMAs and the transform warps' dS stores (tmD) have read it.
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
-__global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0>
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC,
-                   const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
-  static_assert(!XF || (PAIR && sizeof(Elem) == 2 && A_MN == 0 &&
-                        (EPI == EPI_STORE || EPI == EPI_ACCUM)),
-                "operand transform: bf16 2-CTA pairs, K-major A, store or accumulate");
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
@@ -299,7 +250,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   constexpr uint32_t kIdesc =
       idesc_dense(ElemTraits<Elem>::kFmt, kBM * kCtas, kBN, A_MN, B_MN);
   // copies of each CTA complete on its own barriers (else on the leader's)
-  constexpr bool kLocalCopies = XF || !PAIR;
+  constexpr bool kLocalCopies = !PAIR;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -307,8 +258,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint8_t* staging = smem + kRingBytes + kBarrierRegion;  // 1024-B aligned
   uint64_t* empty_bar = full_bar + kNS;
-  uint64_t* ready_bar = empty_bar + kNS;  // XF: stage transformed in both CTAs
-  uint64_t* tfull_bar = ready_bar + kNS;
+  uint64_t* tfull_bar = empty_bar + kNS;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -326,8 +276,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], XF ? 1 + 4 : 1);  // MMA commit (+ each transform warp)
-      mbar_init(&ready_bar[s], 4 * kCtas);        // one arrival per transform warp
+      mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -426,9 +375,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           const uint32_t s = consumed % kNS;
           const uint32_t ph = (consumed / kNS) & 1u;
-          const bool got = XF ? wait_bar(&ready_bar[s], ph, ctl, kPark)
-                              : wait_bar(&full_bar[s], ph, ctl, kPark);
-          if (!got) {
+          if (!wait_bar(&full_bar[s], ph, ctl, kPark)) {
             ok = false;
             break;
           }
@@ -477,82 +424,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else if (XF && warp >= 6) {
-    // ------------------------------------------------------------ operand transform
-    // Warp xw of the four scales rows 32 xw .. 32 xw + 31 of this CTA's A stage
-    // (logit rows m0 + xt), lane = row, with the row's scale for the stage's
-    // 256-column tile kept in a register and loaded one tile (4 stages) ahead.
-    // The rows written are read only by this CTA's tensor core (each CTA of a
-    // pair supplies its own 128 rows of A), so the proxy fence and a CTA-scope
-    // arrival order them before the leader issues the MMAs.  With p.xf_store,
-    // the unit of output column tile xw mod tiles_n also stores the warp's 32
-    // formed rows to the dS chunk (so every row is stored once and the stores
-    // spread over the column tiles); a stored stage is released for refilling
-    // one stage later, once its store has read it.
-    const int xw = warp - 6;
-    const int xt = xw * 32 + lane;  // 0 .. 127
-    uint32_t n = 0;
-    bool ok = true;
-    int pend = -1;  // stage whose store may still be reading it (lane 0)
-    // the dS chunk is read back only by the next kernel: keep it from evicting
-    // the e and W tiles that this kernel's other column tiles re-read from L2
-    const uint64_t ds_policy = l2_policy_evict_first();
-    for (int t = unit; t < total_tiles && ok; t += units) {
-      const UnitRange ur = unit_range(t, p);
-      int tm, tn;
-      tile_coords(ur.tile, p, tm, tn);
-      const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;
-      const int row = m0 + xt;
-      const bool live = row < p.xf_rows;
-      const bool store =
-          p.xf_store != 0 && tn == xw % p.tiles_n && m0 + xw * 32 < p.xf_rows;
-      int cur_t = -1, nxt_t = -1;
-      float cur = 0.f, nxt = 0.f;
-      for (int kb = ur.kb0; kb < ur.kb1; ++kb, ++n) {
-        const uint32_t s = n % kNS;
-        const uint32_t ph = (n / kNS) & 1u;
-        const int k0 = kb * kBKe;
-        if (live && (k0 >> 8) != cur_t) {  // entering a new 256-column tile
-          cur_t = k0 >> 8;
-          cur = (nxt_t == cur_t) ? nxt : __ldg(p.xf_sc + static_cast<int64_t>(cur_t) * p.xf_ld + row);
-          nxt_t = cur_t + 1;
-          if (nxt_t * 256 < p.num_kb * kBKe)  // prefetch the next tile's scale
-            nxt = __ldg(p.xf_sc + static_cast<int64_t>(nxt_t) * p.xf_ld + row);
-        }
-        if (!wait_bar(&full_bar[s], ph, ctl, true)) {
-          ok = false;
-          break;
-        }
-        uint8_t* rows = smem + s * kSBytes + xw * 32 * kRowBytes;  // this warp's 4 KB
-        if (live) xf_row(rows + lane * kRowBytes, lane & 7, __float2bfloat162_rn(cur));
-        fence_proxy_async_smem();  // generic writes -> the tensor core's and TMA's reads
-        __syncwarp();
-        if (lane == 0) {
-          if (store) {
-            tma_store_2d_hint(&tmD, rows, k0, m0 + xw * 32, ds_policy);
-            bulk_commit();
-          }
-          mbar_arrive_cluster(mapa_shared(&ready_bar[s], 0));
-          if (pend >= 0) {  // the previous stored stage: its store has read it
-            if (store) bulk_wait_read_1();
-            else bulk_wait_read_0();
-            mbar_arrive(&empty_bar[pend]);
-            pend = -1;
-          }
-          if (store) pend = static_cast<int>(s);
-          else mbar_arrive(&empty_bar[s]);
-        }
-      }
-    }
-    if (lane == 0) {
-      if (ok && pend >= 0) {
-        bulk_wait_read_0();
-        mbar_arrive(&empty_bar[pend]);
-      }
-      bulk_wait_all();  // the dS stores have landed before exit
-    }
-    __syncwarp();
-  } else if (warp < 4) {
+  } else {
     // ------------------------------------------------------------ epilogue
     // Each warp stages its 32 rows x 32 columns of output in shared memory
     // (two buffers, swizzled to match the output map) and one lane issues a TMA
@@ -648,7 +520,32 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
-        const int gstart = gi;  // first cached entry of this tile (for the dS transform)
+        // Teacher-hidden student pass (tbuf given): the teacher's stored tile
+        // t~ - mt gives, per column, w = 2^((t~ - mt) log2 e) and t~ - s~; the
+        // tile's sums A = sum w (t~ - s~) and U = sum 2^(x - max) (s~ - t~) are
+        // formed in pass 2 from fp32 values.  The teacher values of a 32-column
+        // slab are loaded one slab ahead (slab 0 before pass 1) so that their
+        // latency overlaps the work on the previous slab.
+        const bool hid = p.tbuf != nullptr && rv;
+        const float* trow = hid ? p.tbuf + static_cast<int64_t>(grow) * p.tld : nullptr;
+        auto load_t = [&](int cb, float(&tv)[32]) {
+          const int nv = p.cols_valid - cb;
+          if (nv >= 32) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 t4 = __ldg(reinterpret_cast<const float4*>(trow + cb) + j);
+              tv[4 * j] = t4.x;
+              tv[4 * j + 1] = t4.y;
+              tv[4 * j + 2] = t4.z;
+              tv[4 * j + 3] = t4.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) tv[i] = i < nv ? __ldg(trow + cb + i) : 0.f;
+          }
+        };
+        float tcur[32];
+        if (hid) load_t(col0, tcur);
         // Pass 1: the row's maximum over this tile (base-2 units) and the
         // cached entries' cross term, from the fp32 accumulator.
 #pragma unroll 1
@@ -672,17 +569,10 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
         }
-        // Pass 2: sum of 2^(x - max) and the stored values.  STORE_SHIFTED
-        // stores s~ - max: the entries that carry the probability mass sit near
-        // 0, where the stored value's rounding error vanishes; readers add the
-        // maximum back from the tile statistics.  STORE_EXP stores the
-        // exponentials 2^(x - max) in (0, 1].
-        // Teacher-hidden student pass (tbuf given): the teacher's stored tile
-        // t~ - mt gives, per column, w = 2^((t~ - mt) log2 e) and t~ - s~; the
-        // tile's sums A = sum w (t~ - s~) and U = sum 2^(x - max) (s~ - t~) are
-        // formed here from fp32 values.
-        const bool hid = p.tbuf != nullptr && rv;
-        const float* trow = hid ? p.tbuf + static_cast<int64_t>(grow) * p.tld : nullptr;
+        // Pass 2: sum of 2^(x - max) and the stored values, s~ - max: the
+        // entries that carry the probability mass sit near 0, where the stored
+        // value's rounding error vanishes; readers add the maximum back from
+        // the tile statistics.
         const float mt = hid ? __ldg(&p.tpart[static_cast<int64_t>(grow) * p.tiles_n + tn].x) *
                                    kLn2f
                              : 0.f;
@@ -698,46 +588,34 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
           const int cb = col0 + c * 32;
           const int nvalid = p.cols_valid - cb;
           if (nvalid <= 0) continue;
-          uint32_t e[32];
+          float e[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x = i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
-            se += x;
-            e[i] = __float_as_uint(x);
+            e[i] = i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
+            se += e[i];
           }
           if (hid) {
-            float tv[32];
-            if (nvalid >= 32) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 t4 = __ldg(reinterpret_cast<const float4*>(trow + cb) + j);
-                tv[4 * j] = t4.x;
-                tv[4 * j + 1] = t4.y;
-                tv[4 * j + 2] = t4.z;
-                tv[4 * j + 3] = t4.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) tv[i] = i < nvalid ? __ldg(trow + cb + i) : 0.f;
-            }
+            float tnxt[32];
+            const bool more = c + 1 < kBN / 32 && nvalid > 32;
+            if (more) load_t(cb + 32, tnxt);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               if (i < nvalid) {
-                const float d = (tv[i] + mt) - __uint_as_float(v[i]) * rscale;  // t~ - s~
-                A = fmaf(ex2_approx(tv[i] * kLog2e), d, A);
-                U = fmaf(__uint_as_float(e[i]), -d, U);
+                const float d = (tcur[i] + mt) - __uint_as_float(v[i]) * rscale;  // t~ - s~
+                A = fmaf(ex2_approx(tcur[i] * kLog2e), d, A);
+                U = fmaf(e[i], -d, U);
               }
             }
+            if (more) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) tcur[i] = tnxt[i];
+            }
           }
-          if (p.store == STORE_EXP)
-            store_box(e, 1.f, 0.f, cb, row0, false, false, warp_rows);
-          else if (p.store == STORE_SHIFTED)
-            store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
+          if (p.store) store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] =
-              p.tbuf != nullptr ? make_float4(mx, se, A, U)
-                                : make_float4(mx, se, cross, __int_as_float(gstart));
+              p.tbuf != nullptr ? make_float4(mx, se, A, U) : make_float4(mx, se, cross, 0.f);
       } else if (EPI == EPI_DLOGITS) {
         float coef = 0.f, cm = 0.f, l2 = 0.f;
         const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;

@@ -39,11 +39,14 @@ def _need(t, name, dtype=None, device=None):
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
                  Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0,
-                 v_begin=0, V_total=0):
+                 v_begin=0, V_total=0, keep_last_chunk=False):
     """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive).
     T: a number, or a float32 tensor [N] of per-token temperatures.
     v_begin, V_total: W (and Wt) are rows [v_begin, v_begin + V) of a V_total-row
-    head (vocabulary-parallel calls only)."""
+    head (vocabulary-parallel calls only).
+    keep_last_chunk: kl_fwd leaves the last chunk's logits in its workspace for a
+    following kl_bwd on the same workspace and inputs (no recompute of that
+    chunk)."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
     dev = H.device
@@ -74,6 +77,7 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
     p.reverse_weight = float(reverse_weight)
     p.v_begin = int(v_begin)
     p.V_total = int(V_total)
+    p.keep_last_chunk = 1 if keep_last_chunk else 0
     keep = [H, W, mask, T_row]
     if Ht is not None:
         _need(Ht, "Ht", H.dtype, dev)
@@ -153,6 +157,8 @@ def kl_bwd(H, W, lse_s, lse_t=None, *, grad_loss=None, dW=None, accumulate_dW=Fa
            workspace=None, **kw):
     """Backward with logits recomputed per chunk.  grad_loss: device scalar
     tensor (default 1).  Returns dict(dH, dW)."""
+    if kw.get("keep_last_chunk") and workspace is None:
+        raise ValueError("keep_last_chunk: pass the workspace of the kl_fwd call")
     p, keep = make_problem(H, W, **kw)
     dev = H.device
     ws = workspace if workspace is not None else alloc_workspace(p, L.KL_ENTRY_BWD, dev)
@@ -182,16 +188,26 @@ class _FusedKL(torch.autograd.Function):
                               else out["lse_s"])
         ctx.kw = kw
         ctx.hidden = out["lse_t"] is not None
+        # with keep_last_chunk the workspace carries the last chunk's logits to
+        # the backward (autograd refuses a backward whose H or W changed in place)
+        ctx.ws = out["workspace"] if kw.get("keep_last_chunk") else None
         return out["loss"]
 
     @staticmethod
     def backward(ctx, g):
         H, W, lse_s, lse_t = ctx.saved_tensors
         out = kl_bwd(H, W, lse_s, lse_t if ctx.hidden else None, grad_loss=g.reshape(()),
-                     **ctx.kw)
+                     workspace=ctx.ws, **ctx.kw)
+        ctx.ws = None
         return out["dH"], out["dW"].to(W.dtype), None
 
 
-def fused_kl_loss(H, W, **kw):
-    """Differentiable loss (w.r.t. H and W) via kl_fwd / kl_bwd."""
-    return _FusedKL.apply(H, W, kw)
+def fused_kl_loss(H, W, *, keep_last_chunk=True, **kw):
+    """Differentiable loss (w.r.t. H and W) via kl_fwd / kl_bwd.
+
+    keep_last_chunk (default): the forward's last chunk of logits (one chunk,
+    at most chunk_tokens x V values) stays allocated until the backward, which
+    then recomputes every chunk but that one -- none when N <= chunk_tokens.
+    False: the backward recomputes every chunk and nothing is held between the
+    two passes beyond the per-row log-sum-exps."""
+    return _FusedKL.apply(H, W, dict(kw, keep_last_chunk=keep_last_chunk))

@@ -132,6 +132,17 @@ typedef struct kl_problem {
   int64_t V_total;           /* vocabulary-parallel calls: rows of the whole
                                 head; 0 or V for the other calls.  Cache ids are
                                 always ids of the whole vocabulary.              */
+  int32_t keep_last_chunk;   /* kl_fwd / kl_bwd only, 0 or 1.  1: kl_fwd leaves
+                                the last token chunk's logits and statistics in
+                                the workspace and a following kl_bwd on the same
+                                workspace and the same, unchanged inputs starts
+                                from them instead of recomputing that chunk's
+                                projection (with N <= chunk_tokens, no recompute
+                                at all).  The workspace is then the same size for
+                                every entry (kl_workspace_bytes of FWD_BWD), so
+                                kl_fwd's workspace grows by one chunk of logits,
+                                held until kl_bwd.  Must be 0 for the other
+                                calls (KL_ERR_ARG).                              */
 } kl_problem;
 
 /* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if
@@ -146,8 +157,9 @@ int kl_fwd(const kl_problem* p, void* ws, size_t ws_bytes, float* loss, float* l
            float* lse_t, float* row_loss, void* stream);
 
 /* Backward, recomputing each chunk's logits from H and W (output-head gradient
- * checkpointing, §3 "Fused chunked KL").  lse_s (and lse_t in HIDDEN mode) come
- * from kl_fwd on the same inputs.  grad_loss is a DEVICE pointer to the
+ * checkpointing, §3 "Fused chunked KL") -- except, with keep_last_chunk, the
+ * last chunk, whose logits kl_fwd left in the same workspace (it is processed
+ * first).  lse_s (and lse_t in HIDDEN mode) come from kl_fwd on the same inputs.  grad_loss is a DEVICE pointer to the
  * incoming scalar gradient g.  Writes dH [N, d]; writes dW [V, d] fp32, or adds
  * to it when accumulate_dW != 0.  Tensor work: 6 N d V (+ 2 N d_t V). */
 int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,

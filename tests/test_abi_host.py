@@ -137,3 +137,22 @@ def test_cast_host_checks(lib):
     assert L.kl_cast_f32(None, 256, 8, L.KL_DTYPE_BF16, None) == 1
     assert L.kl_cast_f32(260, 256, 8, L.KL_DTYPE_BF16, None) == 4
     assert L.kl_cast_f32(None, None, 0, L.KL_DTYPE_BF16, None) == 0
+
+
+def test_keep_last_chunk_flag_rules(lib):
+    """keep_last_chunk: 0 or 1; one workspace layout for every entry (kl_fwd
+    leaves the chunk where kl_bwd reads it); refused by the calls that do not
+    pass a chunk from a forward to a backward."""
+    p = _problem()
+    sizes = [L.kl_workspace_bytes(p, e) for e in (0, 1, 2)]
+    p.keep_last_chunk = 1
+    kept = [L.kl_workspace_bytes(p, e) for e in (0, 1, 2)]
+    assert kept[0] == kept[1] == kept[2] == sizes[2]
+    p.keep_last_chunk = 2
+    assert L.kl_workspace_bytes(p, 0) == 0
+    p.keep_last_chunk = 1
+    dummy = 1 << 20
+    rc = L.kl_fwd_bwd(p, dummy, kept[2], 1.0, dummy, None, dummy, dummy, 0, None)
+    assert rc == 10  # KL_ERR_ARG
+    rc = L.kl_fwd_noalloc(p, dummy, dummy, dummy, None, None)
+    assert rc == 10

@@ -128,6 +128,42 @@ def test_split_fwd_then_bwd(mode):
     _check_grad(b["dW"], ref["dW"], "dW")
 
 
+@pytest.mark.parametrize("mode", ["topk", "hidden"])
+@pytest.mark.parametrize("chunk", [128, 0])
+def test_split_keep_last_chunk(mode, chunk):
+    """kl_fwd leaves the last chunk's logits in its workspace and kl_bwd starts
+    from them (several chunks with chunk=128, a single one with the default):
+    the oracle's loss and gradients, and the recompute-everything backward."""
+    w = _small_topk() if mode == "topk" else _small_hidden()
+    beta = 0.3 if mode == "hidden" else 0.0
+    kw = dict(_kw(w, chunk=chunk), reverse_weight=beta)
+    f = ops.kl_fwd(w.H, w.W, keep_last_chunk=True, **kw)
+    g = torch.full((), 0.7, device="cuda")
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"], grad_loss=g, workspace=f["workspace"],
+                   keep_last_chunk=True, **kw)
+    assert ops.status(b["workspace"]) == 0
+    ref = _oracle(w, grad_loss=0.7, reverse_weight=beta)
+    _check_loss(f["loss"].item(), ref["loss"])
+    _check_grad(b["dH"], ref["dH"], "dH")
+    _check_grad(b["dW"], ref["dW"], "dW")
+    r = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"], grad_loss=g, **kw)
+    for k in ("dH", "dW"):
+        a, c = b[k].double(), r[k].double()
+        assert (a - c).abs().max().item() <= 1e-2 * c.abs().max().item(), k
+
+
+def test_split_keep_last_chunk_fp32_tiny():
+    w = wl.tiny().to("cuda")
+    kw = _kw(w, chunk=48)
+    f = ops.kl_fwd(w.H, w.W, keep_last_chunk=True, **kw)
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], grad_loss=torch.full((), 1.1, device="cuda"),
+                   workspace=f["workspace"], keep_last_chunk=True, **kw)
+    ref = _oracle(w, grad_loss=1.1)
+    _check_loss(f["loss"].item(), ref["loss"])
+    _check_grad(b["dH"], ref["dH"], "dH")
+    _check_grad(b["dW"], ref["dW"], "dW")
+
+
 def test_split_fwd_then_bwd_fp32_tiny():
     w = wl.tiny().to("cuda")
     w.mask = torch.ones(w.N, dtype=torch.uint8, device="cuda")
@@ -232,9 +268,7 @@ def test_launch_counter_and_profile():
     ops.kl_fwd_bwd(w.H, w.W, **_kw(w, chunk=128))
     prof = L.kl_profile_end()
     names = {p["name"] for p in prof}
-    # bf16 top-K: dS is formed inside the gradient contractions (no dlogits pass)
-    assert {"gemm_logits_stats", "xf_scales", "gemm_dH", "gemm_dW"} <= names
-    assert "dlogits_topk" not in names
+    assert {"gemm_logits_stats", "gemm_dH", "gemm_dW", "dlogits_topk"} <= names
     assert L.kl_launch_count() - before == sum(p["launches"] for p in prof)
     assert all(p["total_ms"] > 0 for p in prof)
 
