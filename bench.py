@@ -71,6 +71,9 @@ def parse():
                          "shards alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the short runs of the other benchmark configurations that the "
+                         "default single-GPU line carries under 'secondary'")
     ap.add_argument("--cpu-sample", type=int, default=0,
                     help="tokens in the oracle sample (0 = sized to ~10 s)")
     return ap.parse_args()
@@ -474,6 +477,10 @@ def gpu_arm(args):
         "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clk,
         "e2e": e2e,
     }
+    if (ws == 1 and not args.no_secondary and args.workload == "offline_topk" and N == 4096
+            and d == 3072 and args.entry == "fused" and not vocab):
+        del workspace, dH, dW, keep, prob
+        line["secondary"] = secondary_runs(dev, w)
     if not args.no_cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
     if args.workload != "offline_topk":
@@ -497,6 +504,91 @@ def gpu_arm(args):
         executed = step_flops + 2.0 * n_re * V * (d + (w.d_t if w.mode == "hidden" else 0))
         line["executed_tflops_step"] = round(executed * args.steps / (ms / 1e3) / 1e12, 1)
     print(json.dumps(line), flush=True)
+
+
+SECONDARY = [
+    # (name, workload kwargs, entry, timed steps)
+    ("full_vocab_N8192", dict(kind="full_vocab"), "fused", 5),
+    ("packed_long_N32768", dict(kind="packed_long"), "fused", 3),
+    ("scaling_N16384", dict(kind="scaling", N=16384), "fused", 3),
+    ("scaling_N65536", dict(kind="scaling", N=65536), "fused", 2),
+    ("scaling_N262144", dict(kind="scaling", N=262144), "fused", 2),
+    ("offline_topk_N4096_split", dict(kind="offline_topk"), "split", 10),
+]
+
+
+def secondary_runs(dev, main_w):
+    """Short device-timed runs of the other benchmark configurations (the
+    teacher-hidden, packed and scaling workloads, and the split kl_fwd + kl_bwd
+    entry with the last chunk kept, as the autograd path runs it), so that one
+    default run records every configuration.  Each: 2 warm-up steps, then a few
+    steps timed with CUDA events on the launch stream; inputs resident in HBM
+    and larger than L2."""
+    import torch
+
+    from chunked_kl_loss_tma_b200 import _lib, ops
+    from chunked_kl_loss_tma_b200 import workloads as wl
+
+    out = {}
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    for name, spec, entry, steps in SECONDARY:
+        kind = spec["kind"]
+        if kind == "offline_topk":
+            w = main_w
+        elif kind == "full_vocab":
+            w = wl.full_vocab(device=dev)
+        elif kind == "packed_long":
+            w = wl.packed_long(device=dev)
+        else:
+            w = wl.scaling(spec["N"], device=dev)
+        torch.cuda.empty_cache()
+        kw = problem_kwargs(w, 0)
+        prob, keep = ops.make_problem(w.H, w.W, **kw)
+        if entry == "split":
+            prob.keep_last_chunk = 1
+        wsb = ops.workspace_bytes(prob, _lib.KL_ENTRY_FWD_BWD)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        loss = torch.empty((), dtype=torch.float32, device=dev)
+        dH = torch.empty_like(w.H)
+        dW = torch.empty(w.W.shape, dtype=torch.float32, device=dev)
+        lse_s = torch.empty(w.N, dtype=torch.float32, device=dev)
+        g_one = torch.ones((), dtype=torch.float32, device=dev)
+
+        def step():
+            if entry == "split":
+                _lib.check(_lib.kl_fwd(prob, ws.data_ptr(), wsb, loss.data_ptr(), lse_s.data_ptr(),
+                                       None, None, stream), "kl_fwd")
+                _lib.check(_lib.kl_bwd(prob, ws.data_ptr(), wsb, lse_s.data_ptr(), None,
+                                       g_one.data_ptr(), dH.data_ptr(), dW.data_ptr(), 0, stream),
+                           "kl_bwd")
+            else:
+                _lib.check(_lib.kl_fwd_bwd(prob, ws.data_ptr(), wsb, 1.0, loss.data_ptr(), None,
+                                           dH.data_ptr(), dW.data_ptr(), 0, stream), "kl_fwd_bwd")
+
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        status = _lib.kl_status(ws.data_ptr(), stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        flops = 6.0 * w.N * w.d * w.V + (2.0 * w.N * w.d_t * w.V if w.mode == "hidden" else 0.0)
+        out[name] = {"tokens_per_s": round(w.N / (ms / 1e3), 1), "ms_per_step": round(ms, 3),
+                     "steps": steps, "entry": "kl_fwd + kl_bwd (last chunk kept)"
+                     if entry == "split" else "kl_fwd_bwd",
+                     "useful_tflops": round(flops / (ms / 1e3) / 1e12, 1),
+                     "frac_of_spec_2250": round(flops / (ms / 1e3) / 1e12 / 2250.0, 4),
+                     "extra_hbm_gib": round(wsb / 2**30, 4), "status": status,
+                     "loss": round(float(loss.item()), 6)}
+        del prob, keep, ws, dH, dW, lse_s
+        if w is not main_w:
+            del w
+        torch.cuda.empty_cache()
+    return out
 
 
 def _oracle_sample(w, n_tokens):
