@@ -39,8 +39,8 @@
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
 // the 512 columns with one 256 x 512 tile (see the template below).  In the
-// double-buffered variants waiting threads are parked by the hardware between
-// barrier polls rather than spinning.
+// waiting threads are parked by the hardware between barrier polls rather than
+// spinning.
 //
 // Every wait on an mbarrier is bounded (spin_limit clock cycles); when one
 // runs out the CTA records KL_ERR_TIMEOUT in *status and raises the abort flag
@@ -230,13 +230,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
   constexpr int kAccBufs = WIDE ? 1 : 2;              // accumulators in TMEM
-  // Waiting threads let the hardware park them between polls: with two
-  // accumulators the pipeline has slack for the wake-up latency, and the
-  // producer, MMA and epilogue threads stop spinning (logits 10% and dW 3%
-  // faster under the power cap).  The single-accumulator wide tiles keep
-  // spinning: there the wake-up latency is on the critical path (dH 4% slower
-  // when parked).
-  constexpr bool kPark = !WIDE;
+  // Waiting threads let the hardware park them between polls (a 100 ns hint):
+  // the producer, MMA and epilogue threads stop spinning, which under the power
+  // cap made logits 10% and dW 3% faster.  With the short hint the wake-up
+  // latency no longer costs the single-accumulator wide tiles either.
+  constexpr bool kPark = true;
   constexpr int kBRows = kBN / kCtas;                 // B rows per half staged by this CTA
   constexpr int kBBytes = kBRows * kRowBytes;
   constexpr int kSBytes = kATileBytes + kHalves * kBBytes;  // this CTA's stage bytes
