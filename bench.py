@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--entry", default="fused", choices=["fused", "split"],
                     help="fused: kl_fwd_bwd; split: kl_fwd then kl_bwd (the autograd path, "
                          "backward recomputes the logits)")
+    ap.add_argument("--fuse-dlogits", action="store_true",
+                    help="fused entry, bf16 top-K: form dS inside the dH contraction instead of "
+                         "by a pass over the logit chunk (kl_problem.fuse_dlogits)")
     ap.add_argument("--recompute-all", action="store_true",
                     help="--entry split: the backward recomputes every chunk (by default, as "
                          "the autograd path, kl_fwd keeps the last chunk's logits for kl_bwd)")
@@ -228,6 +231,10 @@ def gpu_arm(args):
     kw = problem_kwargs(w, args.chunk)
     if args.reverse_weight > 0:
         kw["reverse_weight"] = args.reverse_weight
+    if args.fuse_dlogits:
+        if args.entry != "fused":
+            raise SystemExit("--fuse-dlogits applies to the fused entry (kl_fwd_bwd)")
+        kw["fuse_dlogits"] = True
     shard = None
     dp_sync = args.dp_sync if (ws > 1 and not vocab) else "none"
     if vocab:
@@ -357,6 +364,8 @@ def gpu_arm(args):
             kw2 = problem_kwargs(w, args.chunk, override=stager.bufs[slot])
             if args.reverse_weight > 0:
                 kw2["reverse_weight"] = args.reverse_weight
+            if args.fuse_dlogits:
+                kw2["fuse_dlogits"] = True
             probs.append(ops.make_problem(stager.bufs[slot]["H"], w.W, **kw2))
         hloss = torch.empty(max(args.steps, 3), dtype=torch.float32).pin_memory()
         cstream = torch.cuda.current_stream(dev)
@@ -478,7 +487,7 @@ def gpu_arm(args):
         "e2e": e2e,
     }
     if (ws == 1 and not args.no_secondary and args.workload == "offline_topk" and N == 4096
-            and d == 3072 and args.entry == "fused" and not vocab):
+            and d == 3072 and args.entry == "fused" and not vocab and not args.fuse_dlogits):
         del workspace, dH, dW, keep, prob
         line["secondary"] = secondary_runs(dev, w)
     if not args.no_cpu_baseline and ws == 1:
@@ -487,6 +496,9 @@ def gpu_arm(args):
         line["metric"] = METRIC + f" [{args.workload}]"
     elif args.d and args.d != 3072:
         line["metric"] = METRIC + f" [d={args.d}]"
+    if args.fuse_dlogits:
+        line["metric"] += " [dS formed in the dH contraction]"
+        line["config"]["fuse_dlogits"] = True
     if args.reverse_weight > 0:
         line["metric"] += f" [reverse KL weight {args.reverse_weight}]"
         line["config"]["reverse_weight"] = args.reverse_weight

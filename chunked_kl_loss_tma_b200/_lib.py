@@ -44,7 +44,7 @@ class KLProblem(ctypes.Structure):
         ("chunk_tokens", ctypes.c_int64), ("normalizer", ctypes.c_float),
         ("reverse_weight", ctypes.c_float), ("T_row", ctypes.c_void_p),
         ("v_begin", ctypes.c_int64), ("V_total", ctypes.c_int64),
-        ("keep_last_chunk", ctypes.c_int32),
+        ("keep_last_chunk", ctypes.c_int32), ("fuse_dlogits", ctypes.c_int32),
     ]
 
 

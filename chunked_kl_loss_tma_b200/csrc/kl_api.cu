@@ -207,6 +207,12 @@ struct Plan {
   // current chunk of H or Ht) and K-major copies W^T [d][Vp], dS^T [V][Cp],
   // H_c^T [d][Cp] for the gradient contractions.
   int64_t Cp = 0;
+  // fuse_dlogits (bf16 top-K): the logits pass stores exponentials, the dH
+  // contraction forms dS from them in shared memory and stores it for dW
+  bool xf = false;
+  int64_t Cx = 0;          // (xf) row stride of the transposed dS scales: C rounded up to 64
+  size_t off_xsc = 0;      // (xf) dS scales [tiles_v][Cx] fp32
+  size_t off_dsbuf = 0;    // (xf) dS chunk [C][Vp] bf16
   size_t off_ubar = 0;     // (hidden) u_bar per chunk row
   int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
   size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
@@ -258,6 +264,7 @@ int validate_shape(const kl_problem* p) {
       (p->reverse_weight > 0.f && p->teacher != KL_TEACHER_HIDDEN))
     return KL_ERR_ARG;
   if (p->keep_last_chunk != 0 && p->keep_last_chunk != 1) return KL_ERR_ARG;
+  if (p->fuse_dlogits != 0 && p->fuse_dlogits != 1) return KL_ERR_ARG;
   if (p->v_begin < 0 || p->V_total < 0 || p->V_total > (int64_t(1) << 31) - 512 ||
       (p->V_total > 0 && p->v_begin + p->V > p->V_total) || (p->V_total == 0 && p->v_begin != 0))
     return KL_ERR_ARG;
@@ -304,6 +311,7 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (pl.C < 1) pl.C = 1;
   pl.Vp = cdiv(p->V, 8) * 8;
   pl.tiles_v = static_cast<int>(cdiv(p->V, kBN));
+  pl.xf = p->fuse_dlogits && pl.eb == 2 && !pl.hidden;
   // student logits / dS chunk: wherever dS is formed (not the forward alone)
   const bool need_sbuf = entry != KL_ENTRY_FWD;
   // tile statistics: every pass that computes them (the top-K backward forms
@@ -323,6 +331,11 @@ Plan make_plan(const kl_problem* p, int entry) {
   if (need_stats && pl.hidden)
     pl.off_pt = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
   if (pl.hidden && entry != KL_ENTRY_FWD) pl.off_ubar = take(static_cast<size_t>(pl.C) * 4);
+  if (pl.xf && entry == KL_ENTRY_FWD_BWD) {
+    pl.Cx = cdiv(pl.C, 64) * 64;
+    pl.off_xsc = take(static_cast<size_t>(pl.tiles_v) * pl.Cx * 4);
+    pl.off_dsbuf = take(buf);  // dS chunk, formed by the dH contraction for dW
+  }
   if (!pl.hidden) {
     pl.off_sidx = take(static_cast<size_t>(pl.C) * p->K * 4);
     pl.off_sq = take(static_cast<size_t>(pl.C) * p->K * 4);
@@ -358,10 +371,11 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
-                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE>;
+                const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops,
+                const CUtensorMap* md = nullptr) {
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -377,7 +391,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(XF ? kGemmThreadsXf : kGemmThreads);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = st;
   if (PAIR) {
@@ -391,7 +405,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md != nullptr ? *md : mc, gp);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
@@ -436,14 +450,15 @@ int prepare_heads(Ctx& c) {
 
 // Logits pass over one chunk: S~ = X_c . Wh^T / T with the tile statistics in
 // `partials`; out != nullptr: s~ - tile max stored into `out` (fp32 when
-// out_f32, else the input type).  tbuf / tpart: the teacher pass's stored tile
-// and statistics (student pass of the teacher-hidden mode: the tile sums A and
-// U go to partials .z / .w).
+// out_f32, else the input type), or with exp_store the bf16 exponentials
+// 2^(s~ log2 e - tile max) (the fused-dS path).  tbuf / tpart: the teacher
+// pass's stored tile and statistics (student pass of the teacher-hidden mode:
+// the tile sums A and U go to partials .z / .w).
 template <typename Elem>
 int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, int64_t Cn,
                 void* out, bool out_f32, float4* partials, const int* sidx,
                 const float* sq, int ktop, const char* name, const float* tbuf = nullptr,
-                const float4* tpart = nullptr) {
+                const float4* tpart = nullptr, bool exp_store = false) {
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   CUtensorMap ma, mb;
@@ -458,6 +473,7 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
       !make_map(&mb, Wh, p->dtype, dx, p->V, dx * sizeof(Elem), kBKe, kBN / 2))
     return KL_ERR_CUDA;
   if (out != nullptr) {
+    out_f32 = out_f32 && !exp_store;
     if (!make_out_map(&mc, out, out_f32 ? KL_DTYPE_F32 : p->dtype, p->V, Cn,
                       c.pl.Vp * (out_f32 ? 4 : sizeof(Elem))))
       return KL_ERR_CUDA;
@@ -469,7 +485,7 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.tiles_n = c.pl.tiles_v;
   gp.num_kb = static_cast<int>(cdiv(dx, kBKe));
   gp.m_fastest = 1;
-  gp.store = out != nullptr;
+  gp.store = out == nullptr ? STORE_NONE : exp_store ? STORE_EXP : STORE_SHIFTED;
   gp.out_f32 = out_f32 ? 1 : 0;
   gp.rows_valid = static_cast<int>(Cn);
   gp.cols_valid = static_cast<int>(p->V);
@@ -594,17 +610,28 @@ int gemm_dlogits(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* lse_s, co
 
 // dH_c = dS . W and dW (+)= dS^T . H_c for chunk rows [c0, c0 + Cn) from the
 // chunk buffer dS.  dH_f32: write dH as fp32 (a vocabulary shard's partial sum)
-// whatever Elem is.
-template <typename Elem>
-int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
-               bool dH_f32 = false) {
-  if (sizeof(Elem) == 4)
-    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
+// whatever Elem is.  XF = 1: the buffer holds the logits pass's exponentials,
+// patched at the cached columns (xf_patch_kernel); the dH contraction forms
+// dS = scale * e in shared memory with the per-(tile, row) scales xf_sc and
+// stores it to the workspace's dS chunk, which the dW contraction reads.
+template <typename Elem, int XF>
+int gemm_grads_bf16(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+                    bool dH_f32, const float* xf_sc) {
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   constexpr int kMNe = kRowBytes / sizeof(Elem);
   const int64_t d = p->d;
   const uint64_t ldS = c.pl.Vp * sizeof(Elem);
+  Elem* dS_formed = XF ? reinterpret_cast<Elem*>(c.ws + c.pl.off_dsbuf) : dS;
+  CUtensorMap md;  // XF: the dS chunk written by the dH contraction, 64 x 32 boxes
+  if (XF && !make_map(&md, dS_formed, p->dtype, p->V, Cn, ldS, kBKe, 32)) return KL_ERR_CUDA;
+  auto set_xf = [&](GemmParams& gp) {
+    if (!XF) return;
+    gp.xf_sc = xf_sc;
+    gp.xf_ld = c.pl.Cx;
+    gp.xf_rows = static_cast<int>(Cn);
+    gp.xf_store = 1;
+  };
   // dH_c = dS . W : A = dS [Cn, V] K-major, B = W as [d, V] MN-major.  When the
   // output has too few tiles to fill the GPU, V is split into ksplit parts whose
   // fp32 partial products are summed in a fixed order afterwards.
@@ -622,6 +649,7 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
     gp.cols_valid = static_cast<int>(d);
     gp.status = &c.sc->status;
     gp.spin_limit = spin_limit();
+    set_xf(gp);
     int ks = choose_ksplit(static_cast<int64_t>(gp.tiles_m) * gp.tiles_n, gp.num_kb, c.sms / 2);
     if (ks > c.pl.ksplit_dh) ks = c.pl.ksplit_dh;
     if (ks > 1) {
@@ -636,8 +664,9 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, part, KL_DTYPE_F32, d, static_cast<uint64_t>(ks) * rows_pad, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
-                                                             gp, 2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
       LaunchScope ls("splitk_reduce", c.st, 0,
                      (4.0 * ks + (dH_f32 ? 4.0 : sizeof(Elem))) * Cn * d);
       if (dH_f32)
@@ -653,22 +682,24 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<float*>(dH) + c0 * d, KL_DTYPE_F32, d, Cn, d * 4))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
-                                                             gp, 2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_ACCUM, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
     } else {
       CUtensorMap mc;
       if (!make_out_map(&mc, static_cast<uint8_t*>(dH) + c0 * d * sizeof(Elem), p->dtype, d, Cn,
                         d * sizeof(Elem)))
         return KL_ERR_CUDA;
-      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide>("gemm_dH", c.st, c.sms, ma, mb, mc,
-                                                             gp, 2.0 * Cn * p->V * d)));
+      KL_TRY((launch_gemm<Elem, 0, 1, EPI_STORE, 1, kDhWide, XF>("gemm_dH", c.st, c.sms, ma, mb,
+                                                                 mc, gp, 2.0 * Cn * p->V * d,
+                                                                 XF ? &md : nullptr)));
     }
   }
   // dW (+)= dS^T . H_c : A = dS^T [V, Cn] MN-major, B = H_c as [d, Cn] MN-major.
   {
     CUtensorMap ma, mb, mc;
     const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * d * sizeof(Elem);
-    if (!make_map(&ma, dS, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
+    if (!make_map(&ma, dS_formed, p->dtype, p->V, Cn, ldS, kMNe, kBKe) ||
         !make_map(&mb, hc, p->dtype, d, Cn, d * sizeof(Elem), kMNe, kBKe) ||
         !make_out_map(&mc, dW, KL_DTYPE_F32, d, p->V, d * 4))
       return KL_ERR_CUDA;
@@ -686,6 +717,19 @@ int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, in
                                                   2.0 * Cn * p->V * d)));
   }
   return KL_OK;
+}
+
+// dH_f32: write dH as fp32 (a vocabulary shard's partial sum) whatever Elem is.
+// xf_sc != nullptr: the fused-dS path (bf16), dS formed in dH's operand path.
+template <typename Elem>
+int gemm_grads(Ctx& c, Elem* dS, int64_t c0, int64_t Cn, void* dH, float* dW, int beta,
+               bool dH_f32 = false, const float* xf_sc = nullptr) {
+  if (sizeof(Elem) == 4)
+    return gemm_grads_f32(c, reinterpret_cast<float*>(dS), c0, Cn, dH, dW, beta);
+  using B = __nv_bfloat16;
+  B* b = reinterpret_cast<B*>(dS);
+  return xf_sc != nullptr ? gemm_grads_bf16<B, 1>(c, b, c0, Cn, dH, dW, beta, dH_f32, xf_sc)
+                          : gemm_grads_bf16<B, 0>(c, b, c0, Cn, dH, dW, beta, dH_f32, nullptr);
 }
 
 int launch_count_valid(Ctx& c) {
@@ -785,6 +829,35 @@ int launch_dlogits_full(Ctx& c, Elem* S, const float* Tt, int64_t c0, int64_t Cn
       p->T_row ? p->T_row + c0 : nullptr, p->reverse_weight,
       reinterpret_cast<const float4*>(c.ws + c.pl.off_ps),
       reinterpret_cast<const float4*>(c.ws + c.pl.off_pt), c.pl.tiles_v);
+  return KL_LAUNCHED();
+}
+
+// dS from the stored exponentials of chunk rows [c0, c0 + Cn) (top-K, bf16):
+// the cached columns' corrections folded into the buffer S, then the
+// transposed per-(tile, row) scales.  lse: the whole problem's rows.  Returns
+// the scales for gemm_grads.
+int launch_xf_prep(Ctx& c, __nv_bfloat16* S, int64_t c0, int64_t Cn, const float* lse,
+                   const float* g_dev, float g_host, const float** xf_sc) {
+  const kl_problem* p = c.p;
+  const float4* part = reinterpret_cast<const float4*>(c.ws + c.pl.off_ps);
+  const float2* rinfo = reinterpret_cast<const float2*>(c.ws + c.pl.off_rinfo);
+  const uint8_t* mask = p->mask ? p->mask + c0 : nullptr;
+  const float* T_row = p->T_row ? p->T_row + c0 : nullptr;
+  float* sc_out = reinterpret_cast<float*>(c.ws + c.pl.off_xsc);
+  {
+    LaunchScope ls("xf_patch", c.st, 0, static_cast<double>(Cn) * p->K * 16);
+    xf_patch_kernel<<<static_cast<unsigned>(cdiv(Cn, 8)), 256, 0, c.st>>>(
+        S, c.pl.Vp, part, c.pl.tiles_v, static_cast<int>(Cn), static_cast<int>(p->V), lse + c0,
+        mask, rinfo, reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
+        reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K, c.sc, g_dev, g_host, c.invT,
+        T_row);
+    KL_TRY(KL_LAUNCHED());
+  }
+  LaunchScope ls("xf_scales", c.st, 0, static_cast<double>(Cn) * c.pl.tiles_v * 20);
+  xf_scales_kernel<<<static_cast<unsigned>(cdiv(Cn, 32)), 256, 0, c.st>>>(
+      part, c.pl.tiles_v, static_cast<int>(Cn), lse + c0, mask, rinfo, c.sc, g_dev, g_host,
+      c.invT, T_row, sc_out, c.pl.Cx);
+  *xf_sc = sc_out;
   return KL_LAUNCHED();
 }
 
@@ -952,8 +1025,15 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
       KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
-                               "gemm_logits_stats"));
+                               "gemm_logits_stats", nullptr, nullptr, c.pl.xf));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
+      if (c.pl.xf) {  // fuse_dlogits: dS formed inside the dH contraction
+        const float* xsc = nullptr;
+        KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
+                              &xsc));
+        KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, false, xsc));
+        continue;
+      }
       KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
     } else {
       float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
@@ -996,7 +1076,7 @@ int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
     KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                              reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                              reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
-                             "gemm_logits_stats"));
+                             "gemm_logits_stats", nullptr, nullptr, c.pl.xf));
     return launch_row_stats(c, ps, Cn, stats, 0, true);
   }
   float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
@@ -1052,8 +1132,15 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sum
   const int beta = (accumulate || k > 0) ? 1 : 0;
   KL_TRY(launch_vp_merge(c, c0, Cn, stats_all, P, rank, lse_user, rl));
   if (!c.pl.hidden) {
-    KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
-    KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
+    if (c.pl.xf) {  // fuse_dlogits: dS formed inside the dH contraction
+      const float* xsc = nullptr;
+      KL_TRY(launch_xf_prep(c, reinterpret_cast<__nv_bfloat16*>(S), c0, Cn, lse_s, nullptr, g,
+                            &xsc));
+      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true, xsc));
+    } else {
+      KL_TRY(launch_dlogits_topk<Elem>(c, S, c0, Cn, lse_s, nullptr, g, ps));
+      KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
+    }
   } else {
     // this shard's A, U (its row-loss share) and u_bar, the sum of every shard's
     // U when the reverse KL needs it (its sums came through the second exchange)
@@ -1090,6 +1177,7 @@ size_t kl_workspace_bytes(const kl_problem* p, int entry) {
 
 int kl_fwd(const kl_problem* p, void* ws, size_t ws_bytes, float* loss, float* lse_s,
            float* lse_t, float* row_loss, void* stream) {
+  if (p != nullptr && p->fuse_dlogits) return KL_ERR_ARG;
   Ctx c;
   KL_TRY(begin(p, KL_ENTRY_FWD, ws, ws_bytes, stream, c));
   if (loss == nullptr || (p->N > 0 && lse_s == nullptr) ||
@@ -1102,6 +1190,7 @@ int kl_fwd(const kl_problem* p, void* ws, size_t ws_bytes, float* loss, float* l
 int kl_bwd(const kl_problem* p, void* ws, size_t ws_bytes, const float* lse_s,
            const float* lse_t, const float* grad_loss, void* dH, float* dW, int accumulate_dW,
            void* stream) {
+  if (p != nullptr && p->fuse_dlogits) return KL_ERR_ARG;
   Ctx c;
   KL_TRY(begin(p, KL_ENTRY_BWD, ws, ws_bytes, stream, c));
   if (dW == nullptr || grad_loss == nullptr ||
@@ -1285,7 +1374,7 @@ int noalloc_scratch(uint8_t** out) {
 
 extern "C" int kl_fwd_noalloc(const kl_problem* p, float* loss, float* lse_s, float* row_loss,
                               int* status, void* stream) {
-  if (p != nullptr && p->keep_last_chunk) return KL_ERR_ARG;
+  if (p != nullptr && (p->keep_last_chunk || p->fuse_dlogits)) return KL_ERR_ARG;
   KL_TRY(validate(p));
   if (!whole_head(p)) return KL_ERR_ARG;
   if (p->dtype != KL_DTYPE_BF16 || p->teacher != KL_TEACHER_TOPK) return KL_ERR_DTYPE;

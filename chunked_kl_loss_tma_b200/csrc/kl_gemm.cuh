@@ -1,8 +1,9 @@
 // kl_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for the three
 // contractions of the fused KL loss, with the loss arithmetic fused into the
-// epilogue ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits
-// and a Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection
-// is integrated into the loss and each logit chunk is transient).
+// epilogue and, optionally, into the dH contraction's operand path
+// ("Efficient Knowledge Distillation for LLMs: Offline Top-K Logits and a
+// Fused Chunked KL Loss", §3 "Fused chunked KL": the output projection is
+// integrated into the loss and each logit chunk is transient).
 //
 //   C[M, N] = A[M, K] . B[N, K]^T   (bf16 -> kind::f16, fp32 -> kind::tf32;
 //                                     fp32 accumulation in TMEM)
@@ -11,7 +12,10 @@
 //              max and sum of 2^(s~ log2 e - max) and the cross term
 //              sum_i q_i s~_{idx_i} of the cached top-K entries that fall in
 //              the tile (gathered from the fp32 accumulator).  Optionally
-//              stores s~ - max (natural units; fp32 or the input type).  In
+//              stores s~ - max (store = 1; natural units; fp32 or the input
+//              type) or the exponentials 2^(s~ log2 e - max) themselves
+//              (store = 2), which the dH contraction then scales into dS as its
+//              operand stages arrive (XF, the opt-in fused-dS path).  In
 //              the teacher-hidden mode the student pass also reads the
 //              teacher tile (stored fp32 by the teacher pass) and forms the
 //              tile's sums sum p_t (t~ - s~) and sum p_s (s~ - t~) from fp32.
@@ -35,7 +39,15 @@
 //   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
-//   warp 5     TMEM allocator + MMA issuer (one thread).
+//   warp 5     TMEM allocator + MMA issuer (one thread);
+//   warps 6-9  (XF = 1 only, dH) operand transform: turn the A stage -- the
+//              stored exponentials e = 2^(s~ log2 e - tile max) of a logit
+//              chunk, already corrected at the cached entries -- into
+//              dS = scale(row, tile) * e in shared memory before the MMAs read
+//              it, and store the formed stage as the dS chunk that the dW
+//              contraction then reads.  This is the dlogits step of the loss
+//              without its own pass over HBM (measured slower than that pass
+//              on B200 at d >= 2048, so it is opt-in).
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
 // the 512 columns with one 256 x 512 tile (see the template below).  In the
@@ -64,6 +76,7 @@ constexpr int kATileBytes = kBM * kRowBytes;
 constexpr int kBTileBytes = kBN * kRowBytes;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmThreads = 192;
+constexpr int kGemmThreadsXf = 320;  // + four operand-transform warps
 constexpr int kTmemCols = 2 * kBN;
 constexpr int kRingBytes = kStages * kStageBytes;          // 192 KB operand ring
 constexpr int kBarrierRegion = 1024;                        // barriers, TMEM slot, flags
@@ -83,12 +96,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2f = 0.6931471805599453f;
 
 enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3 };
+// EPI_STATS store modes
+enum { STORE_NONE = 0, STORE_SHIFTED = 1, STORE_EXP = 2 };
 
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
-  int store;           // STATS: store s~ - tile max through the output map (0 = statistics only)
-  int out_f32;         // STATS with store: the output map holds fp32
+  int store;           // STATS: STORE_NONE / STORE_SHIFTED / STORE_EXP
+  int out_f32;         // STATS, STORE_SHIFTED: the output map holds fp32
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
   float scale;         // STATS / DLOGITS: 1 / T
@@ -103,6 +118,13 @@ struct GemmParams {
   const float* tbuf;
   int64_t tld;
   const float4* tpart;
+  // XF: scale of dS per (256-column tile, logit row), [tiles][xf_ld] fp32
+  // (xf_ld a multiple of 64), so that dS = scale * e for the stored e
+  const float* xf_sc;
+  int64_t xf_ld;
+  int xf_rows;         // logit rows (tokens) that exist
+  int xf_store;        // XF: store each formed dS stage through the fourth map (the
+                       // dS chunk for dW); each row by one output column tile
   // DLOGITS: per-row lse (natural units), (m, .) per row, mask, and the scalars
   // of c = g / (n T): the loss normaliser n, and g (device pointer or value)
   const float* lse;
@@ -214,18 +236,46 @@ __device__ __forceinline__ void store_vec<float>(float* dst, const float* v) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// XF: one 128-byte row of a dS operand stage (64 bf16 values of one logit row
+// within one 256-column tile), x -> x * scale in place with packed bf16x2
+// multiplies (scale rounded to bf16: with the product's rounding, 2^-8
+// relative error per entry).  The chunks are visited in the row's swizzled
+// order (chunk j at position j ^ sw) so that the 32 rows a warp's lanes touch
+// at once hit all 32 banks.
+__device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 scale2) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint4* cp = reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4));
+    uint4 u = *cp;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __hmul2(h[i], scale2);
+    *cp = u;
+  }
+}
+
 // WIDE = 1 (2-CTA pairs, store / accumulate epilogues): each work unit is a
 // 256 x 512 output tile computed as two N = 256 MMAs per K step that share the
 // A stage, so a CTA pulls 25% fewer operand bytes from L2 per MMA.  Both halves
 // fill all 512 TMEM columns, so there is a single accumulator: the next unit's
 // MMAs wait for the epilogue (worth it where units are long, as in dH).
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// XF = 1 (dH: 2-CTA pairs, bf16, K-major A, store / accumulate epilogues): the
+// A operand is a stage of stored exponentials that the transform warps turn
+// into dS.  Each CTA's copies then complete on its own barriers (the transform
+// warps of both CTAs wait for them), the MMA issuer waits for the transforms
+// of both CTAs on a third ring of barriers, and a stage is refilled only after
+// the MMAs and the transform warps' dS stores (tmD) have read it.
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
+__global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
+  static_assert(!XF || (PAIR && sizeof(Elem) == 2 && A_MN == 0 &&
+                        (EPI == EPI_STORE || EPI == EPI_ACCUM)),
+                "operand transform: bf16 2-CTA pairs, K-major A, store or accumulate");
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
@@ -248,7 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr uint32_t kIdesc =
       idesc_dense(ElemTraits<Elem>::kFmt, kBM * kCtas, kBN, A_MN, B_MN);
   // copies of each CTA complete on its own barriers (else on the leader's)
-  constexpr bool kLocalCopies = !PAIR;
+  constexpr bool kLocalCopies = XF || !PAIR;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -256,7 +306,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint8_t* staging = smem + kRingBytes + kBarrierRegion;  // 1024-B aligned
   uint64_t* empty_bar = full_bar + kNS;
-  uint64_t* tfull_bar = empty_bar + kNS;
+  uint64_t* ready_bar = empty_bar + kNS;  // XF: stage transformed in both CTAs
+  uint64_t* tfull_bar = ready_bar + kNS;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -274,7 +325,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&empty_bar[s], XF ? 1 + 4 : 1);  // MMA commit (+ each transform warp)
+      mbar_init(&ready_bar[s], 4 * kCtas);        // one arrival per transform warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -373,7 +425,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
           const uint32_t s = consumed % kNS;
           const uint32_t ph = (consumed / kNS) & 1u;
-          if (!wait_bar(&full_bar[s], ph, ctl, kPark)) {
+          const bool got = XF ? wait_bar(&ready_bar[s], ph, ctl, kPark)
+                              : wait_bar(&full_bar[s], ph, ctl, kPark);
+          if (!got) {
             ok = false;
             break;
           }
@@ -422,7 +476,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (XF && warp >= 6) {
+    // ------------------------------------------------------------ operand transform
+    // Warp xw of the four scales rows 32 xw .. 32 xw + 31 of this CTA's A stage
+    // (logit rows m0 + xt), lane = row, with the row's scale for the stage's
+    // 256-column tile kept in a register and loaded one tile (4 stages) ahead.
+    // The rows written are read only by this CTA's tensor core (each CTA of a
+    // pair supplies its own 128 rows of A), so the proxy fence and a CTA-scope
+    // arrival order them before the leader issues the MMAs.  With p.xf_store,
+    // the unit of output column tile xw mod tiles_n also stores the warp's 32
+    // formed rows to the dS chunk (so every row is stored once and the stores
+    // spread over the column tiles); a stored stage is released for refilling
+    // one stage later, once its store has read it.
+    const int xw = warp - 6;
+    const int xt = xw * 32 + lane;  // 0 .. 127
+    uint32_t n = 0;
+    bool ok = true;
+    int pend = -1;  // stage whose store may still be reading it (lane 0)
+    // the dS chunk is read back only by the next kernel: keep it from evicting
+    // the e and W tiles that this kernel's other column tiles re-read from L2
+    const uint64_t ds_policy = l2_policy_evict_first();
+    for (int t = unit; t < total_tiles && ok; t += units) {
+      const UnitRange ur = unit_range(t, p);
+      int tm, tn;
+      tile_coords(ur.tile, p, tm, tn);
+      const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;
+      const int row = m0 + xt;
+      const bool live = row < p.xf_rows;
+      const bool store =
+          p.xf_store != 0 && tn == xw % p.tiles_n && m0 + xw * 32 < p.xf_rows;
+      int cur_t = -1, nxt_t = -1;
+      float cur = 0.f, nxt = 0.f;
+      for (int kb = ur.kb0; kb < ur.kb1; ++kb, ++n) {
+        const uint32_t s = n % kNS;
+        const uint32_t ph = (n / kNS) & 1u;
+        const int k0 = kb * kBKe;
+        if (live && (k0 >> 8) != cur_t) {  // entering a new 256-column tile
+          cur_t = k0 >> 8;
+          cur = (nxt_t == cur_t) ? nxt : __ldg(p.xf_sc + static_cast<int64_t>(cur_t) * p.xf_ld + row);
+          nxt_t = cur_t + 1;
+          if (nxt_t * 256 < p.num_kb * kBKe)  // prefetch the next tile's scale
+            nxt = __ldg(p.xf_sc + static_cast<int64_t>(nxt_t) * p.xf_ld + row);
+        }
+        if (!wait_bar(&full_bar[s], ph, ctl, true)) {
+          ok = false;
+          break;
+        }
+        uint8_t* rows = smem + s * kSBytes + xw * 32 * kRowBytes;  // this warp's 4 KB
+        if (live) xf_row(rows + lane * kRowBytes, lane & 7, __float2bfloat162_rn(cur));
+        fence_proxy_async_smem();  // generic writes -> the tensor core's and TMA's reads
+        __syncwarp();
+        if (lane == 0) {
+          if (store) {
+            tma_store_2d_hint(&tmD, rows, k0, m0 + xw * 32, ds_policy);
+            bulk_commit();
+          }
+          mbar_arrive_cluster(mapa_shared(&ready_bar[s], 0));
+          if (pend >= 0) {  // the previous stored stage: its store has read it
+            if (store) bulk_wait_read_1();
+            else bulk_wait_read_0();
+            mbar_arrive(&empty_bar[pend]);
+            pend = -1;
+          }
+          if (store) pend = static_cast<int>(s);
+          else mbar_arrive(&empty_bar[s]);
+        }
+      }
+    }
+    if (lane == 0) {
+      if (ok && pend >= 0) {
+        bulk_wait_read_0();
+        mbar_arrive(&empty_bar[pend]);
+      }
+      bulk_wait_all();  // the dS stores have landed before exit
+    }
+    __syncwarp();
+  } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
     // Each warp stages its 32 rows x 32 columns of output in shared memory
     // (two buffers, swizzled to match the output map) and one lane issues a TMA
@@ -567,10 +696,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
           }
         }
-        // Pass 2: sum of 2^(x - max) and the stored values, s~ - max: the
-        // entries that carry the probability mass sit near 0, where the stored
-        // value's rounding error vanishes; readers add the maximum back from
-        // the tile statistics.
+        // Pass 2: sum of 2^(x - max) and the stored values.  STORE_SHIFTED
+        // stores s~ - max: the entries that carry the probability mass sit near
+        // 0, where the stored value's rounding error vanishes; readers add the
+        // maximum back from the tile statistics.  STORE_EXP stores the
+        // exponentials 2^(x - max) in (0, 1].
         const float mt = hid ? __ldg(&p.tpart[static_cast<int64_t>(grow) * p.tiles_n + tn].x) *
                                    kLn2f
                              : 0.f;
@@ -609,7 +739,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int i = 0; i < 32; ++i) tcur[i] = tnxt[i];
             }
           }
-          if (p.store) store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
+          if (p.store == STORE_SHIFTED) {
+            store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
+          } else if (p.store == STORE_EXP) {
+            uint32_t eb[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) eb[i] = __float_as_uint(e[i]);
+            store_box(eb, 1.f, 0.f, cb, row0, false, false, warp_rows);
+          }
         }
         if (rv && p.partials != nullptr)
           p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] =

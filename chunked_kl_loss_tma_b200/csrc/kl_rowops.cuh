@@ -341,6 +341,72 @@ __global__ void dlogits_topk_kernel(Elem* __restrict__ S, int64_t ld, int V,
   }
 }
 
+// dS from the stored exponentials (bf16 top-K, the opt-in fused-dS path).  The
+// logits pass stores e_j = 2^(s~_j log2 e - M) with M the (row, 256-column tile) maximum
+// (base 2), so the dense part of dS_j = c (m p_s,j - q_j [j in S]) is
+// scale * e_j with
+//   scale = c m 2^(max(M - lse log2 e, -64)),
+// where c = g / (n T) (0 on masked rows).  The floor at 2^-64 keeps scale a
+// normal float when a tile lies far below the row's maximum; the dense part it
+// then adds, at most c m 2^-64 per entry, is far below any entry that matters.
+// The correction -c q_j at a cached column is folded into the stored value
+// itself (xf_patch_kernel), so that dS = scale * e everywhere and the dH
+// contraction applies one factor per (row, tile) to its operand stages.
+__device__ __forceinline__ float xf_scale(float cm, float M2, float l2) {
+  return cm * ex2_approx(fmaxf(M2 - l2, -64.f));
+}
+
+// One warp per row, lanes over the K cached entries: e_j <- e_j - c q_j / scale
+// at each cached column j of this head (bf16 stored exponentials in S, row
+// stride ld), with scale as xf_scale for j's tile.  Reads the logits pass's
+// tile maxima (part.x); masked rows and rows without cache mass keep e (their
+// scale is 0).
+__global__ void xf_patch_kernel(__nv_bfloat16* __restrict__ S, int64_t ld,
+                                const float4* __restrict__ part, int tiles_n, int rows, int V,
+                                const float* __restrict__ lse, const uint8_t* __restrict__ mask,
+                                const float2* __restrict__ rowinfo,
+                                const int* __restrict__ sidx, const float* __restrict__ sq,
+                                int K, const Scalars* sc, const float* g_dev, float g_host,
+                                float invT, const float* __restrict__ T_row) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const float c = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
+  const float cm = c * rowinfo[row].x;
+  if (cm == 0.f) return;
+  const float l2 = lse[row] * kLog2e;
+  const int* ri = sidx + static_cast<int64_t>(row) * K;
+  const float* rq = sq + static_cast<int64_t>(row) * K;
+  __nv_bfloat16* srow = S + static_cast<int64_t>(row) * ld;
+  for (int i = lane; i < K; i += 32) {
+    const int j = ri[i];  // in [0, V): a cached column of this head; else empty or elsewhere
+    if (static_cast<unsigned>(j) >= static_cast<unsigned>(V)) continue;
+    const float scale =
+        xf_scale(cm, part[static_cast<int64_t>(row) * tiles_n + (j >> 8)].x, l2);
+    srow[j] = __float2bfloat16_rn(__bfloat162float(srow[j]) - c * rq[i] / scale);
+  }
+}
+
+// Scales of dS (xf_scale) for the chunk's rows, transposed for the gradient
+// contractions: sc_out[t * ld + row] for tile t.  A block covers 32 rows (lane
+// = row, so the writes of each tile are contiguous) and its warps share the
+// tiles.
+__global__ void xf_scales_kernel(const float4* __restrict__ part, int tiles_n, int rows,
+                                 const float* __restrict__ lse, const uint8_t* __restrict__ mask,
+                                 const float2* __restrict__ rowinfo, const Scalars* sc,
+                                 const float* g_dev, float g_host, float invT,
+                                 const float* __restrict__ T_row, float* __restrict__ sc_out,
+                                 int64_t ld) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 32 + lane;
+  if (row >= rows) return;
+  const float cm = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row) * rowinfo[row].x;
+  const float l2 = lse[row] * kLog2e;
+  const float4* pr = part + static_cast<int64_t>(row) * tiles_n;
+  for (int t = warp; t < tiles_n; t += blockDim.x >> 5)
+    sc_out[static_cast<int64_t>(t) * ld + row] = xf_scale(cm, pr[t].x, l2);
+}
+
 // Teacher-hidden mode, one warp per row: from the tile statistics of the two
 // logits passes -- student (max2, sumexp2, A_tile, U_tile) and teacher (max2,
 // sumexp2, ., .), with A_tile = sum 2^(t - mt) (t~ - s~) and

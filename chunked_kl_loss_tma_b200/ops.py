@@ -39,14 +39,16 @@ def _need(t, name, dtype=None, device=None):
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
                  Ht=None, Wt=None, chunk_tokens=0, normalizer=0.0, reverse_weight=0.0,
-                 v_begin=0, V_total=0, keep_last_chunk=False):
+                 v_begin=0, V_total=0, keep_last_chunk=False, fuse_dlogits=False):
     """Fill a kl_problem from tensors.  Returns (problem, tensors kept alive).
     T: a number, or a float32 tensor [N] of per-token temperatures.
     v_begin, V_total: W (and Wt) are rows [v_begin, v_begin + V) of a V_total-row
     head (vocabulary-parallel calls only).
     keep_last_chunk: kl_fwd leaves the last chunk's logits in its workspace for a
     following kl_bwd on the same workspace and inputs (no recompute of that
-    chunk)."""
+    chunk).
+    fuse_dlogits: kl_fwd_bwd / kl_vp_* form dS inside the dH contraction (bf16
+    top-K) instead of by a pass over the logit chunk."""
     if not isinstance(H, torch.Tensor) or not H.is_cuda:
         raise ValueError("H must be a CUDA tensor")
     dev = H.device
@@ -78,6 +80,7 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
     p.v_begin = int(v_begin)
     p.V_total = int(V_total)
     p.keep_last_chunk = 1 if keep_last_chunk else 0
+    p.fuse_dlogits = 1 if fuse_dlogits else 0
     keep = [H, W, mask, T_row]
     if Ht is not None:
         _need(Ht, "Ht", H.dtype, dev)

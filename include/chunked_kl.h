@@ -143,6 +143,17 @@ typedef struct kl_problem {
                                 kl_fwd's workspace grows by one chunk of logits,
                                 held until kl_bwd.  Must be 0 for the other
                                 calls (KL_ERR_ARG).                              */
+  int32_t fuse_dlogits;      /* kl_fwd_bwd / kl_vp_* only, 0 or 1; bf16 top-K mode
+                                (ignored otherwise).  1: dS is formed inside the
+                                dH contraction's operand path instead of by a
+                                pass over the logit chunk (§3 "Fused chunked
+                                KL": logits turned into gradients on the way
+                                into the gradient projections).  Same results
+                                up to rounding; on B200 it measured slower than
+                                the separate pass at d >= 2048 (default 0).
+                                The workspace grows by one chunk of dS.  kl_fwd,
+                                kl_bwd and kl_fwd_noalloc refuse it
+                                (KL_ERR_ARG).                                    */
 } kl_problem;
 
 /* Bytes of workspace that entry (KL_ENTRY_*) needs for this problem, or 0 if

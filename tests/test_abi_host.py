@@ -156,3 +156,22 @@ def test_keep_last_chunk_flag_rules(lib):
     assert rc == 10  # KL_ERR_ARG
     rc = L.kl_fwd_noalloc(p, dummy, dummy, dummy, None, None)
     assert rc == 10
+
+
+def test_fuse_dlogits_flag_rules(lib):
+    """fuse_dlogits: 0 or 1; the fused pass's workspace grows by one chunk of dS
+    (bf16 top-K only); kl_fwd, kl_bwd and the no-allocation forward refuse it."""
+    p = _problem()
+    base = L.kl_workspace_bytes(p, 2)
+    p.fuse_dlogits = 1
+    assert L.kl_workspace_bytes(p, 2) >= base + 4096 * 128256 * 2
+    p.dtype = 1  # fp32 inputs keep the dlogits pass: no extra buffer
+    assert L.kl_workspace_bytes(p, 2) == L.kl_workspace_bytes(_problem(dtype=1), 2)
+    p.dtype = 0
+    p.fuse_dlogits = 2
+    assert L.kl_workspace_bytes(p, 2) == 0
+    p.fuse_dlogits = 1
+    dummy = 1 << 20
+    assert L.kl_fwd(p, dummy, base, dummy, dummy, None, None, None) == 10  # KL_ERR_ARG
+    assert L.kl_bwd(p, dummy, base, dummy, None, dummy, dummy, dummy, 0, None) == 10
+    assert L.kl_fwd_noalloc(p, dummy, dummy, dummy, None, None) == 10

@@ -144,6 +144,26 @@ def test_offline_topk_4096_full_oracle_pass():
     _identities(w, out)
 
 
+def test_offline_topk_4096_fused_dlogits():
+    """The bench workload with dS formed inside the dH contraction: the oracle's
+    sampled rows, the identities and the separate-pass result."""
+    w = wl.offline_topk(device="cuda", seed=9)
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, fuse_dlogits=True, **_kw(w))
+    assert ops.status(out["workspace"]) == 0
+    rows = _rows(w.N, None, n_random=16, seed=9)
+    _check_rows(w, out, rows, w.N)
+    _loss_is_mean_of_rows(out, w.N)
+    _identities(w, out)
+    # The two paths round dS differently (the fused one rounds its bf16 scale and
+    # then the product); both are held to the gradient tolerance against the
+    # oracle above, and to the same bound against each other.
+    plain = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w))
+    assert torch.equal(out["loss"], plain["loss"])
+    for k in ("dH", "dW"):
+        a, c = out[k].double(), plain[k].double()
+        assert (a - c).abs().max().item() <= 2e-2 * c.abs().max().item(), k
+
+
 def test_offline_topk_4096_split_forward_backward():
     """kl_fwd then kl_bwd (backward recomputes the logits and forms dS in the
     GEMM epilogue) against the oracle's sampled rows and the fused path."""

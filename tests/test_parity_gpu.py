@@ -177,6 +177,53 @@ def test_split_fwd_then_bwd_fp32_tiny():
     _check_grad(b["dW"], ref["dW"], "dW")
 
 
+@pytest.mark.parametrize("partial", [True, False])
+@pytest.mark.parametrize("chunk", [128, 0])
+def test_fused_dlogits_path(partial, chunk):
+    """fuse_dlogits: the logits pass stores exponentials, the cached entries'
+    corrections are folded into them, and dH forms dS in shared memory and
+    stores it for dW -- against the oracle, with a mask, several chunks and a
+    ragged tail in every dimension, and against the separate dlogits pass."""
+    w = _small_topk(partial=partial)
+    out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=1.7, want_row_loss=True, fuse_dlogits=True,
+                         **_kw(w, chunk))
+    assert ops.status(out["workspace"]) == 0
+    ref = _oracle(w, grad_loss=1.7)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    plain = ops.kl_fwd_bwd(w.H, w.W, grad_loss=1.7, want_row_loss=True, **_kw(w, chunk))
+    assert torch.equal(out["row_loss"], plain["row_loss"])
+    for k in ("dH", "dW"):  # differently rounded dS: the gradient tolerance
+        a, c = out[k].double(), plain[k].double()
+        assert (a - c).abs().max().item() <= GRAD_FRAC * c.abs().max().item(), k
+
+
+@pytest.mark.parametrize("case", ["K_equals_V", "per_token_T", "accumulate"])
+def test_fused_dlogits_edge_cases(case):
+    if case == "K_equals_V":
+        w = wl.make_topk("kvx", N=96, d=64, V=320, K=320, d_t=32, T=1.0, dtype=torch.bfloat16,
+                         w_std=0.1, tw_std=0.2, seed=23).to("cuda")
+        kw = _kw(w)
+    elif case == "per_token_T":
+        Tr = _per_token_T(300, 29)
+        w = wl.make_topk("pttx", N=300, d=200, V=5003, K=16, d_t=64, T=Tr, dtype=torch.bfloat16,
+                         w_std=0.05, tw_std=0.1, seed=29).to("cuda")
+        kw = _kw(w, chunk=128)
+    else:
+        w = _small_topk(seed=21)
+        kw = _kw(w, chunk=64)
+    base = torch.randn(w.W.shape, device="cuda", dtype=torch.float32)
+    acc = case == "accumulate"
+    out = ops.kl_fwd_bwd(w.H, w.W, dW=base.clone() if acc else None, accumulate_dW=acc,
+                         fuse_dlogits=True, **kw)
+    assert ops.status(out["workspace"]) == 0
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"] - base if acc else out["dW"], ref["dW"], "dW")
+
+
 def test_autograd_function_matches_oracle():
     w = _small_topk(N=160, V=2100, masked=False)
     H = w.H.clone().requires_grad_(True)
@@ -271,6 +318,11 @@ def test_launch_counter_and_profile():
     assert {"gemm_logits_stats", "gemm_dH", "gemm_dW", "dlogits_topk"} <= names
     assert L.kl_launch_count() - before == sum(p["launches"] for p in prof)
     assert all(p["total_ms"] > 0 for p in prof)
+    L.kl_profile_begin()
+    ops.kl_fwd_bwd(w.H, w.W, fuse_dlogits=True, **_kw(w, chunk=128))
+    names = {p["name"] for p in L.kl_profile_end()}
+    assert {"gemm_logits_stats", "xf_patch", "xf_scales", "gemm_dH", "gemm_dW"} <= names
+    assert "dlogits_topk" not in names
 
 
 def test_bitwise_deterministic_across_calls():

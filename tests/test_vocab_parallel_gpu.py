@@ -95,6 +95,18 @@ def test_topk_shards_match_oracle(partial, layout):
     _check_all(out, _oracle(w, grad_loss=1.7))
 
 
+@pytest.mark.parametrize("layout", ["P2", "P3_ragged"])
+def test_topk_shards_fused_dlogits(layout):
+    """Shards with dS formed inside each shard's dH contraction (fuse_dlogits),
+    including a 3-row shard and boundaries inside tiles."""
+    w = _topk(seed=37)
+    shards = TOPK_SHARDS[layout]
+    P = 2 if shards is None else len(shards)
+    out = vp.emulate(w.H, w.W, P, shards=shards, grad_loss=1.1, want_row_loss=True,
+                     want_lse=True, fuse_dlogits=True, **_kw(w, chunk=128))
+    _check_all(out, _oracle(w, grad_loss=1.1))
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_hidden_shards_match_oracle(dtype):
     w = _hidden(dtype=dtype)

@@ -21,9 +21,9 @@ CHILD = textwrap.dedent("""
     w = wl.make_topk("wd", N=600, d=256, V=9000, K=16, d_t=64, T=1.0,
                      dtype=torch.bfloat16, w_std=0.05, tw_std=0.1, seed=41).to("cuda")
     codes = []
-    for _ in range(2):
+    for fuse in (False, True):  # the separate dlogits pass, and dS formed inside dH
         out = ops.kl_fwd_bwd(w.H, w.W, topk_idx=w.topk_idx, topk_logit=w.topk_logit,
-                             teacher_lse=w.teacher_lse, chunk_tokens=256)
+                             teacher_lse=w.teacher_lse, chunk_tokens=256, fuse_dlogits=fuse)
         codes.append(ops.status(out["workspace"]))
     torch.cuda.synchronize()
     ok = float(torch.ones(1000, device="cuda").sum().item()) == 1000.0
