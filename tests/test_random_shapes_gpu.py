@@ -1,0 +1,99 @@
+"""Seeded random problems through the CUDA path against the fp64 oracle.
+
+Each case draws its sizes and options from one seed: the token count N, the
+widths d and d_t (multiples of 8), the vocabulary V (often not a multiple of 8
+or of the 256-column tile), the cache width K (up to V), the teacher mode, bf16
+or fp32 inputs, a scalar or per-token temperature, a random mask, the chunk
+size, partial mass or renormalised teacher probabilities, a reverse-KL weight in
+the teacher-hidden mode, and the entry: the fused pass (with or without dS
+formed inside the dH contraction) or kl_fwd followed by kl_bwd (with or without
+the kept last chunk).  Tolerances as in the other parity tests: loss relative
+error <= 1e-3 (plus 1e-6 absolute, for losses that are 0), gradients max-abs
+error <= 2e-2 * max|oracle gradient|."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_tma_b200 import ops
+from chunked_kl_loss_tma_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+CASES = 48
+
+
+def _draw(seed):
+    rng = np.random.default_rng(1000 + seed)
+    mode = "hidden" if rng.random() < 0.35 else "topk"
+    dtype = torch.float32 if rng.random() < 0.2 else torch.bfloat16
+    N = int(rng.integers(1, 700))
+    d = 8 * int(rng.integers(1, 70))
+    V = int(rng.choice([int(rng.integers(1, 300)), int(rng.integers(300, 9000))]))
+    K = int(rng.integers(1, min(V, 96) + 1))
+    d_t = 8 * int(rng.integers(1, 40))
+    per_token = rng.random() < 0.3
+    T = float(rng.uniform(0.5, 3.0))
+    chunk = int(rng.choice([0, 64, 200, 512]))
+    masked = rng.random() < 0.5
+    partial = rng.random() < 0.6
+    beta = float(rng.choice([0.0, 0.0, 0.3, 1.0])) if mode == "hidden" else 0.0
+    entry = str(rng.choice(["fused", "fused", "split", "split_keep"]))
+    fuse = bool(mode == "topk" and dtype == torch.bfloat16 and entry == "fused" and
+                rng.random() < 0.5)
+    g = float(rng.uniform(0.3, 2.0))
+    Tr = None
+    if per_token:
+        Tr = torch.from_numpy(rng.uniform(0.5, 3.0, size=N).astype(np.float32))
+    w_std = float(rng.uniform(0.03, 0.3))
+    if mode == "topk":
+        w = wl.make_topk(f"rand{seed}", N=N, d=d, V=V, K=K, d_t=d_t, T=Tr if per_token else T,
+                         dtype=dtype, w_std=w_std, tw_std=float(rng.uniform(0.05, 0.3)),
+                         seed=2000 + seed, partial_mass=partial)
+    else:
+        w = wl.make_hidden(f"randh{seed}", N=N, d=d, d_t=d_t, V=V, T=Tr if per_token else T,
+                           dtype=dtype, w_std=w_std, tw_std=float(rng.uniform(0.05, 0.3)),
+                           seed=2000 + seed)
+    if masked:
+        w.mask = torch.from_numpy((rng.random(N) > 0.25).astype(np.uint8))
+    opts = dict(chunk=chunk, beta=beta, entry=entry, fuse=fuse, g=g)
+    return w.to("cuda"), opts
+
+
+def _kw(w, opts):
+    kw = dict(T=w.T, mask=w.mask, chunk_tokens=opts["chunk"], reverse_weight=opts["beta"])
+    if w.mode == "topk":
+        kw.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        kw.update(Ht=w.Ht, Wt=w.Wt)
+    return kw
+
+
+@pytest.mark.parametrize("seed", range(CASES))
+def test_random_problem_matches_oracle(seed):
+    w, o = _draw(seed)
+    kw = _kw(w, o)
+    if o["entry"] == "fused":
+        out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=o["g"], fuse_dlogits=o["fuse"], **kw)
+        loss, dH, dW, wss = out["loss"], out["dH"], out["dW"], [out["workspace"]]
+    else:
+        keep = o["entry"] == "split_keep"
+        f = ops.kl_fwd(w.H, w.W, keep_last_chunk=keep, **kw)
+        b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"],
+                       grad_loss=torch.full((), o["g"], device="cuda"),
+                       workspace=f["workspace"] if keep else None, keep_last_chunk=keep, **kw)
+        loss, dH, dW, wss = f["loss"], b["dH"], b["dW"], [f["workspace"], b["workspace"]]
+    assert all(ops.status(ws) == 0 for ws in wss)
+    args = dict(T=w.T, mask=w.mask, mode=w.mode, grad_loss=o["g"], reverse_weight=o["beta"])
+    if w.mode == "topk":
+        args.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        args.update(Ht=w.Ht, Wt=w.Wt)
+    ref = oracle.kl_loss(w.H, w.W, **args)
+    case = f"seed {seed}: N={w.N} d={w.d} V={w.V} {w.mode} {w.dtype} {o}"
+    assert abs(loss.item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-6, \
+        (case, loss.item(), ref["loss"])
+    for name, got in (("dH", dH), ("dW", dW)):
+        r = ref[name]
+        err = np.max(np.abs(got.double().cpu().numpy() - r))
+        assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
