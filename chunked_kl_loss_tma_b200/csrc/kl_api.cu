@@ -214,11 +214,9 @@ struct Plan {
   size_t off_xsc = 0;      // (xf) dS scales [tiles_v][Cx] fp32
   size_t off_dsbuf = 0;    // (xf) dS chunk [C][Vp] bf16
   size_t off_ubar = 0;     // (hidden) u_bar per chunk row
-  size_t off_tscr = 0;     // (hidden) per-CTA fp32 teacher values of the dual logits pass
-  bool t_f32 = false;      // (hidden) teacher chunk for the dS pass in fp32 (else bf16)
   int ksplit_dh = 1;       // K-parts of the dH contraction (fp32 partials + reduce)
   size_t off_dhp = 0;      // dH partials [ksplit_dh][C][d] fp32
-  size_t off_wr = 0, off_wtr = 0, off_xr = 0, off_xtr = 0, off_wT = 0, off_sT = 0, off_hT = 0;
+  size_t off_wr = 0, off_wtr = 0, off_xr = 0, off_wT = 0, off_sT = 0, off_hT = 0;
 };
 
 // Sizes, dtypes and scalar arguments (no pointers).
@@ -327,15 +325,8 @@ Plan make_plan(const kl_problem* p, int entry) {
   };
   const size_t buf = static_cast<size_t>(pl.C) * pl.Vp * pl.eb;
   if (need_sbuf) pl.off_sbuf = take(buf);
-  // teacher logits chunk (t~ - tile max) for the dS pass: bf16 for the forward
-  // KL, whose p_t tolerates it as p_s does; fp32 with a reverse-KL weight, whose
-  // term p_s (s~ - t~ - u_bar) needs s~ - t~ to fp32 accuracy wherever p_s is
-  // large, however far t~ is from its tile maximum there.  The loss sums use
-  // the fp32 values that the dual logits pass keeps per CTA.
-  pl.t_f32 = pl.eb == 4 || p->reverse_weight > 0.f;
-  if (pl.hidden && need_sbuf)
-    pl.off_tbuf = take(static_cast<size_t>(pl.C) * pl.Vp * (pl.t_f32 ? 4 : pl.eb));
-  if (pl.hidden) pl.off_tscr = take(static_cast<size_t>(kDualMaxCtas) * kDualScratchBytes);
+  // teacher logits chunk, fp32: the student pass forms the loss sums from it
+  if (pl.hidden) pl.off_tbuf = take(static_cast<size_t>(pl.C) * pl.Vp * 4);
   if (need_stats) pl.off_ps = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
   if (need_stats && pl.hidden)
     pl.off_pt = take(static_cast<size_t>(pl.C) * pl.tiles_v * sizeof(float4));
@@ -364,12 +355,10 @@ Plan make_plan(const kl_problem* p, int entry) {
                         p->d * 4);
   }
   if (pl.eb == 4) {
+    const int64_t dmax = (pl.hidden && p->d_t > p->d) ? p->d_t : p->d;
     pl.off_wr = take(static_cast<size_t>(p->V) * p->d * 4);
-    pl.off_xr = take(static_cast<size_t>(pl.C) * p->d * 4);
-    if (pl.hidden) {  // the dual pass reads both rounded chunks
-      pl.off_wtr = take(static_cast<size_t>(p->V) * p->d_t * 4);
-      pl.off_xtr = take(static_cast<size_t>(pl.C) * p->d_t * 4);
-    }
+    if (pl.hidden) pl.off_wtr = take(static_cast<size_t>(p->V) * p->d_t * 4);
+    pl.off_xr = take(static_cast<size_t>(pl.C) * dmax * 4);
   }
   if (pl.eb == 4 && entry != KL_ENTRY_FWD) {
     pl.Cp = cdiv(pl.C, 4) * 4;
@@ -385,8 +374,7 @@ Plan make_plan(const kl_problem* p, int entry) {
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops,
-                const CUtensorMap* md = nullptr, const CUtensorMap* me = nullptr,
-                const CUtensorMap* mf = nullptr) {
+                const CUtensorMap* md = nullptr) {
   auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
@@ -399,8 +387,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   }
   const int tiles = gp.tiles_m * gp.tiles_n * gp.ksplit;  // work units
   const int units = PAIR ? sms / 2 : sms;  // CTA pairs or CTAs, one CTA per SM
-  int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
-  if (EPI == EPI_DUAL && grid > kDualMaxCtas) grid = kDualMaxCtas;  // scratch blocks
+  const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid);
@@ -418,8 +405,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaError_t e;
   {
     LaunchScope ls(name, st, flops, 0);
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md != nullptr ? *md : mc,
-                           me != nullptr ? *me : mc, mf != nullptr ? *mf : mc, gp);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md != nullptr ? *md : mc, gp);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? KL_OK : KL_ERR_CUDA;
 }
@@ -465,11 +451,14 @@ int prepare_heads(Ctx& c) {
 // Logits pass over one chunk: S~ = X_c . Wh^T / T with the tile statistics in
 // `partials`; out != nullptr: s~ - tile max stored into `out` (fp32 when
 // out_f32, else the input type), or with exp_store the bf16 exponentials
-// 2^(s~ log2 e - tile max) (the fused-dS path).
+// 2^(s~ log2 e - tile max) (the fused-dS path).  tbuf / tpart: the teacher
+// pass's stored tile and statistics (student pass of the teacher-hidden mode:
+// the tile sums A and U go to partials .z / .w).
 template <typename Elem>
 int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, int64_t Cn,
                 void* out, bool out_f32, float4* partials, const int* sidx,
-                const float* sq, int ktop, const char* name, bool exp_store = false) {
+                const float* sq, int ktop, const char* name, const float* tbuf = nullptr,
+                const float4* tpart = nullptr, bool exp_store = false) {
   const kl_problem* p = c.p;
   constexpr int kBKe = kRowBytes / sizeof(Elem);
   CUtensorMap ma, mb;
@@ -506,6 +495,9 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.sidx = sidx;
   gp.sq = sq;
   gp.ktop = ktop;
+  gp.tbuf = tbuf;
+  gp.tld = c.pl.Vp;
+  gp.tpart = tpart;
   gp.status = &c.sc->status;
   gp.spin_limit = spin_limit();
   return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, mc, gp,
@@ -826,27 +818,17 @@ int launch_dlogits_topk(Ctx& c, Elem* S, int64_t c0, int64_t Cn, const float* ls
 
 // dS in place over the student buffer, teacher-hidden mode (one CTA per row).
 template <typename Elem>
-int launch_dlogits_full(Ctx& c, Elem* S, const void* Tt, int64_t c0, int64_t Cn,
+int launch_dlogits_full(Ctx& c, Elem* S, const float* Tt, int64_t c0, int64_t Cn,
                         const float* lse_s, const float* lse_t, const float* ubar,
                         const float* g_dev, float g_host) {
   const kl_problem* p = c.p;
-  LaunchScope ls("dlogits_full", c.st, 0,
-                 (2.0 * sizeof(Elem) + (c.pl.t_f32 ? 4.0 : sizeof(Elem))) * Cn * p->V);
-  const unsigned grid = static_cast<unsigned>(Cn);
-  const float4* ps = reinterpret_cast<const float4*>(c.ws + c.pl.off_ps);
-  const float4* pt = reinterpret_cast<const float4*>(c.ws + c.pl.off_pt);
-  const uint8_t* mask = p->mask ? p->mask + c0 : nullptr;
-  const float* T_row = p->T_row ? p->T_row + c0 : nullptr;
-  if (c.pl.t_f32)
-    dlogits_full_kernel<Elem, float><<<grid, kDlogitsFullThreads, 0, c.st>>>(
-        S, static_cast<const float*>(Tt), c.pl.Vp, static_cast<int>(p->V), lse_s + c0,
-        lse_t + c0, ubar, mask, c.sc, g_dev, g_host, c.invT, T_row, p->reverse_weight, ps, pt,
-        c.pl.tiles_v);
-  else
-    dlogits_full_kernel<Elem, Elem><<<grid, kDlogitsFullThreads, 0, c.st>>>(
-        S, static_cast<const Elem*>(Tt), c.pl.Vp, static_cast<int>(p->V), lse_s + c0,
-        lse_t + c0, ubar, mask, c.sc, g_dev, g_host, c.invT, T_row, p->reverse_weight, ps, pt,
-        c.pl.tiles_v);
+  LaunchScope ls("dlogits_full", c.st, 0, (2.0 * sizeof(Elem) + 4.0) * Cn * p->V);
+  dlogits_full_kernel<Elem><<<static_cast<unsigned>(Cn), kDlogitsFullThreads, 0, c.st>>>(
+      S, Tt, c.pl.Vp, static_cast<int>(p->V), lse_s + c0, lse_t + c0, ubar,
+      p->mask ? p->mask + c0 : nullptr, c.sc, g_dev, g_host, c.invT,
+      p->T_row ? p->T_row + c0 : nullptr, p->reverse_weight,
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_ps),
+      reinterpret_cast<const float4*>(c.ws + c.pl.off_pt), c.pl.tiles_v);
   return KL_LAUNCHED();
 }
 
@@ -899,67 +881,21 @@ int launch_hidden_sums(Ctx& c, int64_t c0, int64_t Cn, const float* lse_s_in,
   return KL_LAUNCHED();
 }
 
-// Row tiles of 256 tokens that the dual logits pass keeps in flight at once.
-int kDualGroupM = 16;
-
-// Teacher-hidden logits of one chunk in one launch (EPI_DUAL): per 256 x 256
-// tile the teacher's accumulator (Ht_c . Wt^T), then the student's
-// (H_c . W^T).  Tile statistics of both into the teacher / student partials,
-// the tile sums A and U into the student partials' .z / .w; with `store`,
-// t~ - tile max and s~ - tile max (input type) into the teacher and student
-// buffers for the dS pass.
+// Teacher-hidden logits of one chunk: the teacher pass (fp32 t~ - tile max into
+// the teacher buffer, statistics), then the student pass (statistics and the
+// tile sums A, U formed against the teacher tile; s~ - tile max stored into
+// the student buffer when store_student).
 template <typename Elem>
-int hidden_logits(Ctx& c, int64_t c0, int64_t Cn, bool store) {
+int hidden_logits(Ctx& c, int64_t c0, int64_t Cn, bool store_student) {
   const kl_problem* p = c.p;
-  constexpr int kBKe = kRowBytes / sizeof(Elem);
-  const int64_t eb = sizeof(Elem);
-  const uint8_t* hc = static_cast<const uint8_t*>(p->H) + c0 * p->d * eb;
-  const uint8_t* htc = static_cast<const uint8_t*>(p->Ht) + c0 * p->d_t * eb;
-  if (sizeof(Elem) == 4) {  // tf32: round both chunks of hidden states first
-    float* xr = reinterpret_cast<float*>(c.ws + c.pl.off_xr);
-    float* xtr = reinterpret_cast<float*>(c.ws + c.pl.off_xtr);
-    KL_TRY(launch_round(c, reinterpret_cast<const float*>(hc), p->d, xr, p->d, Cn, p->d));
-    KL_TRY(launch_round(c, reinterpret_cast<const float*>(htc), p->d_t, xtr, p->d_t, Cn,
-                        p->d_t));
-    hc = reinterpret_cast<const uint8_t*>(xr);
-    htc = reinterpret_cast<const uint8_t*>(xtr);
-  }
-  CUtensorMap ma, mb, mc, md, me, mf;
-  if (!make_map(&ma, hc, p->dtype, p->d, Cn, p->d * eb, kBKe, kBM) ||
-      !make_map(&mb, head_W(c), p->dtype, p->d, p->V, p->d * eb, kBKe, kBN / 2) ||
-      !make_map(&md, htc, p->dtype, p->d_t, Cn, p->d_t * eb, kBKe, kBM) ||
-      !make_map(&me, head_Wt(c), p->dtype, p->d_t, p->V, p->d_t * eb, kBKe, kBN / 2))
-    return KL_ERR_CUDA;
-  if (store) {
-    if (!make_out_map(&mc, c.ws + c.pl.off_sbuf, p->dtype, p->V, Cn, c.pl.Vp * eb) ||
-        !make_out_map(&mf, c.ws + c.pl.off_tbuf, c.pl.t_f32 ? KL_DTYPE_F32 : p->dtype, p->V,
-                      Cn, c.pl.Vp * (c.pl.t_f32 ? 4 : eb)))
-      return KL_ERR_CUDA;
-  } else {
-    mc = mb;  // statistics only: the output maps are not used
-    mf = mb;
-  }
-  GemmParams gp{};
-  gp.tiles_m = static_cast<int>(cdiv(Cn, 2 * kBM));
-  gp.tiles_n = c.pl.tiles_v;
-  gp.num_kb = static_cast<int>(cdiv(p->d, kBKe));
-  gp.num_kb_t = static_cast<int>(cdiv(p->d_t, kBKe));
-  gp.m_fastest = 1;
-  gp.group_m = kDualGroupM;
-  gp.store = store ? STORE_SHIFTED : STORE_NONE;
-  gp.store_t = store ? 1 : 0;
-  gp.t_f32 = c.pl.t_f32 ? 1 : 0;
-  gp.rows_valid = static_cast<int>(Cn);
-  gp.cols_valid = static_cast<int>(p->V);
-  gp.scale = c.invT;
-  gp.T_row = p->T_row ? p->T_row + c0 : nullptr;
-  gp.partials = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
-  gp.tpartials = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
-  gp.tscr = reinterpret_cast<float4*>(c.ws + c.pl.off_tscr);
-  gp.status = &c.sc->status;
-  gp.spin_limit = spin_limit();
-  return launch_gemm<Elem, 0, 0, EPI_DUAL, 1>("gemm_logits_dual", c.st, c.sms, ma, mb, mc, gp,
-                                              2.0 * Cn * p->V * (p->d + p->d_t), &md, &me, &mf);
+  float* Tt = reinterpret_cast<float*>(c.ws + c.pl.off_tbuf);
+  float4* ps = reinterpret_cast<float4*>(c.ws + c.pl.off_ps);
+  float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
+  KL_TRY(gemm_logits<Elem>(c, p->Ht, p->d_t, head_Wt(c), c0, Cn, Tt, true, pt,
+                           nullptr, nullptr, 0, "gemm_teacher_logits"));
+  return gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn,
+                           store_student ? c.ws + c.pl.off_sbuf : nullptr, sizeof(Elem) == 4, ps,
+                           nullptr, nullptr, 0, "gemm_logits_stats", Tt, pt);
 }
 
 int launch_finalize(Ctx& c, const float* row_loss, float* loss) {
@@ -1055,8 +991,8 @@ int run_bwd(Ctx& c, const float* lse_s, const float* lse_t, const float* g_dev, 
       if (!kept) KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
       KL_TRY(launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, 1, nullptr, nullptr,
                                 ubar));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, c.ws + c.pl.off_tbuf, c0, Cn, lse_s, lse_t, ubar,
-                                       g_dev, g_host));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                       c0, Cn, lse_s, lse_t, ubar, g_dev, g_host));
     }
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, (accumulate || i > 0) ? 1 : 0));
   }
@@ -1089,7 +1025,7 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
       KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                                reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                                reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
-                               "gemm_logits_stats", c.pl.xf));
+                               "gemm_logits_stats", nullptr, nullptr, c.pl.xf));
       KL_TRY(launch_row_reduce(c, ps, c0, Cn, true, lse_s, rl));
       if (c.pl.xf) {  // fuse_dlogits: dS formed inside the dH contraction
         const float* xsc = nullptr;
@@ -1103,8 +1039,8 @@ int run_fwd_bwd(Ctx& c, float g, float* loss, float* row_loss, void* dH, float* 
       float* ubar = reinterpret_cast<float*>(c.ws + c.pl.off_ubar);
       KL_TRY(hidden_logits<Elem>(c, c0, Cn, true));
       KL_TRY(launch_hidden_sums(c, c0, Cn, nullptr, nullptr, lse_s, lse_t, 1, rl, nullptr, ubar));
-      KL_TRY(launch_dlogits_full<Elem>(c, S, c.ws + c.pl.off_tbuf, c0, Cn, lse_s, lse_t, ubar,
-                                       nullptr, g));
+      KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                       c0, Cn, lse_s, lse_t, ubar, nullptr, g));
     }
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta));
   }
@@ -1140,7 +1076,7 @@ int run_vp_fwd_chunk(Ctx& c, int64_t k, float* stats) {
     KL_TRY(gemm_logits<Elem>(c, p->H, p->d, head_W(c), c0, Cn, S, sizeof(Elem) == 4, ps,
                              reinterpret_cast<const int*>(c.ws + c.pl.off_sidx),
                              reinterpret_cast<const float*>(c.ws + c.pl.off_sq), p->K,
-                             "gemm_logits_stats", c.pl.xf));
+                             "gemm_logits_stats", nullptr, nullptr, c.pl.xf));
     return launch_row_stats(c, ps, Cn, stats, 0, true);
   }
   float4* pt = reinterpret_cast<float4*>(c.ws + c.pl.off_pt);
@@ -1212,8 +1148,8 @@ int run_vp_bwd_chunk(Ctx& c, int64_t k, const float* stats_all, const float* sum
     const bool mixed = p->reverse_weight > 0.f;
     KL_TRY(launch_hidden_sums(c, c0, Cn, lse_s, lse_t, nullptr, nullptr, rank == 0 ? 1 : 0, rl,
                               nullptr, ubar, mixed ? sums_all : nullptr, P));
-    KL_TRY(launch_dlogits_full<Elem>(c, S, c.ws + c.pl.off_tbuf, c0, Cn, lse_s, lse_t, ubar,
-                                     nullptr, g));
+    KL_TRY(launch_dlogits_full<Elem>(c, S, reinterpret_cast<const float*>(c.ws + c.pl.off_tbuf),
+                                     c0, Cn, lse_s, lse_t, ubar, nullptr, g));
     KL_TRY(gemm_grads<Elem>(c, S, c0, Cn, dH, dW, beta, true));
   }
   if (c0 + Cn == p->N) KL_TRY(launch_finalize(c, rl, loss));

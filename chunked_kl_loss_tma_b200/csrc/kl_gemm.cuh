@@ -15,19 +15,10 @@
 //              stores s~ - max (store = 1; natural units; fp32 or the input
 //              type) or the exponentials 2^(s~ log2 e - max) themselves
 //              (store = 2), which the dH contraction then scales into dS as its
-//              operand stages arrive (XF, the opt-in fused-dS path).
-//   EPI_DUAL   teacher-hidden mode, both logit tiles of one 256 x 256 output
-//              tile in one work unit: the teacher tile T = Ht_c . Wt^T
-//              (K = d_t) into TMEM columns 0-255, then the student tile
-//              S = H_c . W^T (K = d) into columns 256-511.  The epilogue takes
-//              the teacher half first: its tile statistics, t~ - max kept in
-//              fp32 in a per-CTA scratch that stays in L2, optionally stored
-//              (fp32 or the input type) for the dS pass, and the columns
-//              released so that the next unit's teacher MMAs overlap the
-//              student half.  The student half then forms its statistics and
-//              the tile sums sum p_t (t~ - s~) and sum p_s (s~ - t~) from the
-//              fp32 accumulator and the fp32 teacher values, and optionally
-//              stores s~ - max.
+//              operand stages arrive (XF, the opt-in fused-dS path).  In
+//              the teacher-hidden mode the student pass also reads the
+//              teacher tile (stored fp32 by the teacher pass) and forms the
+//              tile's sums sum p_t (t~ - s~) and sum p_s (s~ - t~) from fp32.
 //   EPI_STORE  dH_c = dS . W    -> element type of H, clipped to the chunk.
 //   EPI_ACCUM  dW  (+)= dS^T . H_c -> fp32, add-reduced into dW across chunks;
 //              also the fp32 split-K parts of dH.
@@ -47,8 +38,7 @@
 // Roles (192 threads, one CTA per SM, grid-strided over output tiles):
 //   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
-//   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles (for
-//              EPI_DUAL the teacher's K-blocks, then the student's);
+//   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
 //   warp 5     TMEM allocator + MMA issuer (one thread);
 //   warps 6-9  (XF = 1 only, dH) operand transform: turn the A stage -- the
 //              stored exponentials e = 2^(s~ log2 e - tile max) of a logit
@@ -105,39 +95,29 @@ constexpr long long kDrainLimit = 1LL << 31;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2f = 0.6931471805599453f;
 
-enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3, EPI_DUAL = 4 };
-// EPI_DUAL: fp32 teacher values one CTA keeps between the two halves of a unit
-// (128 rows x 256 columns); the launch gives each CTA its own block.
-constexpr int kDualScratchBytes = kBM * kBN * 4;
-constexpr int kDualMaxCtas = 160;  // grid bound of an EPI_DUAL launch
+enum { EPI_STATS = 0, EPI_STORE = 1, EPI_ACCUM = 2, EPI_DLOGITS = 3 };
 // EPI_STATS store modes
 enum { STORE_NONE = 0, STORE_SHIFTED = 1, STORE_EXP = 2 };
 
 struct GemmParams {
   int tiles_m, tiles_n, num_kb;  // tiles_m counts 256-row tiles when PAIR = 1
-  int num_kb_t;        // DUAL: K-blocks of the teacher contraction (num_kb: student)
   int m_fastest;       // raster: consecutive tile ids walk M first (else N first)
-  int group_m;         // with m_fastest: walk M within groups of group_m row tiles,
-                       // one group after the other (0: one group of all rows)
   int store;           // STATS: STORE_NONE / STORE_SHIFTED / STORE_EXP
-                       // (DUAL: STORE_NONE or STORE_SHIFTED for the student tile)
-  int store_t;         // DUAL: store t~ - max through the sixth map
-  int t_f32;           // DUAL: ... in fp32 (else the input type)
   int out_f32;         // STATS, STORE_SHIFTED: the output map holds fp32
   int rows_valid;      // output rows that exist (M extent)
   int cols_valid;      // output columns that exist (N extent)
   float scale;         // STATS / DLOGITS: 1 / T
   const float* T_row;  // STATS / DLOGITS: per-row temperature (chunk rows), or nullptr
   int beta;            // ACCUM: 0 overwrite, 1 accumulate
-  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross, 0);
-                       // DUAL, student: (max2, sumexp2, A, U)
+  float4* partials;    // STATS: [rows][tiles_n] (max2, sumexp2, cross | A, 0 | U)
   const int* sidx;     // STATS gather: [rows][ktop] ascending ids, INT_MAX = empty
   const float* sq;     // STATS gather: [rows][ktop] teacher probabilities
   int ktop;            // STATS gather: entries per row (0 = no gather)
-  // DUAL: the teacher's tile statistics [rows][tiles_n] (max2, sumexp2, 0, 0)
-  // and the scratch, kDualScratchBytes per CTA of the grid
-  float4* tpartials;
-  float4* tscr;
+  // STATS, student pass of the teacher-hidden mode: the teacher tile stored by
+  // the teacher pass (t~ - tile max, fp32, row stride tld) and its statistics
+  const float* tbuf;
+  int64_t tld;
+  const float4* tpart;
   // XF: scale of dS per (256-column tile, logit row), [tiles][xf_ld] fp32
   // (xf_ld a multiple of 64), so that dS = scale * e for the stored e
   const float* xf_sc;
@@ -226,12 +206,8 @@ __device__ __forceinline__ float round_tf32_dev(float x) {
 
 __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm, int& tn) {
   if (p.m_fastest) {
-    const int gm = (p.group_m > 0 && p.group_m < p.tiles_m) ? p.group_m : p.tiles_m;
-    const int g = t / (gm * p.tiles_n);   // group of row tiles
-    const int r = t - g * gm * p.tiles_n;
-    const int rows = min(gm, p.tiles_m - g * gm);  // row tiles in this group
-    tm = g * gm + r % rows;
-    tn = r / rows;
+    tm = t % p.tiles_m;
+    tn = t / p.tiles_m;
   } else {
     tn = t % p.tiles_n;
     tm = t / p.tiles_n;
@@ -289,21 +265,14 @@ __device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 sca
 // warps of both CTAs wait for them), the MMA issuer waits for the transforms
 // of both CTAs on a third ring of barriers, and a stage is refilled only after
 // the MMAs and the transform warps' dS stores (tmD) have read it.
-// EPI_DUAL: tmA / tmB the student operands (H_c, W), tmC the student tile's
-// output map, tmD / tmE the teacher operands (Ht_c, Wt), tmF the teacher
-// tile's output map.  Other epilogues use tmA .. tmD as described above.
 template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
 __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC,
-                   const __grid_constant__ CUtensorMap tmD,
-                   const __grid_constant__ CUtensorMap tmE,
-                   const __grid_constant__ CUtensorMap tmF, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   static_assert(!WIDE || (PAIR && (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "wide tiles: 2-CTA pairs with a store or accumulate epilogue");
-  static_assert(EPI != EPI_DUAL || (PAIR && !A_MN && !B_MN),
-                "dual logits: 2-CTA pairs, K-major operands");
   static_assert(!XF || (PAIR && sizeof(Elem) == 2 && A_MN == 0 &&
                         (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "operand transform: bf16 2-CTA pairs, K-major A, store or accumulate");
@@ -311,8 +280,6 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
   constexpr int kAccBufs = WIDE ? 1 : 2;              // accumulators in TMEM
-  // contractions per work unit (DUAL: teacher into accumulator 0, student into 1)
-  constexpr int kParts = EPI == EPI_DUAL ? 2 : 1;
   // Waiting threads let the hardware park them between polls (a 100 ns hint):
   // the producer, MMA and epilogue threads stop spinning, which under the power
   // cap made logits 10% and dW 3% faster.  With the short hint the wake-up
@@ -373,10 +340,6 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (EPI == EPI_DUAL) {
-      tma_prefetch_desc(&tmD);
-      tma_prefetch_desc(&tmE);
-    }
   }
   if (warp == 5) {
     if (PAIR) {
@@ -395,16 +358,6 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   const uint32_t peer_abort =
       PAIR ? mapa_shared(const_cast<int*>(abort_flag), rank ^ 1u) : 0u;
   const Ctl ctl{p.status, p.spin_limit, abort_flag, peer_abort};
-  // K-blocks of contraction `part` of a unit (DUAL: whole K of each operand pair)
-  auto part_kb = [&](const UnitRange& ur, int part, int& kb0, int& kb1) {
-    if (EPI == EPI_DUAL) {
-      kb0 = 0;
-      kb1 = part == 0 ? p.num_kb_t : p.num_kb;
-    } else {
-      kb0 = ur.kb0;
-      kb1 = ur.kb1;
-    }
-  };
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -417,44 +370,38 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
         tile_coords(ur.tile, p, tm, tn);
         const int m0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM;  // this CTA's A rows
         const int n0 = tn * kTileN + static_cast<int>(rank) * kBRows;     // this CTA's B rows
-        for (int part = 0; part < kParts && ok; ++part) {
-          const CUtensorMap* mapA = (EPI == EPI_DUAL && part == 0) ? &tmD : &tmA;
-          const CUtensorMap* mapB = (EPI == EPI_DUAL && part == 0) ? &tmE : &tmB;
-          int kbb, kbe;
-          part_kb(ur, part, kbb, kbe);
-          for (int kb = kbb; kb < kbe; ++kb) {
-            const uint32_t s = issued % kNS;
-            const uint32_t ph = (issued / kNS) & 1u;
-            if (!wait_bar(&empty_bar[s], ph ^ 1u, ctl, kPark)) {
-              ok = false;
-              break;
-            }
-            uint8_t* a_s = smem + s * kSBytes;
-            uint8_t* b_s = a_s + kATileBytes;
-            if (kLocalCopies) mbar_arrive_expect_tx(&full_bar[s], kSBytes);
-            else if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
-            const uint32_t fb = kLocalCopies ? 0u : mapa_shared(&full_bar[s], 0);
-            const int k0 = kb * kBKe;
-#pragma unroll
-            for (int sl = 0; sl < (A_MN ? kBM / kMNe : 1); ++sl) {
-              void* dst = a_s + sl * kSlabBytes;
-              const int x = A_MN ? m0 + sl * kMNe : k0, y = A_MN ? k0 : m0;
-              if (kLocalCopies) tma_load_2d(mapA, &full_bar[s], dst, x, y);
-              else tma_load_2d_pair(mapA, fb, dst, x, y);
-            }
-#pragma unroll
-            for (int h = 0; h < kHalves; ++h) {
-              const int nh = n0 + h * kBN;  // this CTA's B rows of half h
-#pragma unroll
-              for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
-                void* dst = b_s + h * kBBytes + sl * kSlabBytes;
-                const int x = B_MN ? nh + sl * kMNe : k0, y = B_MN ? k0 : nh;
-                if (kLocalCopies) tma_load_2d(mapB, &full_bar[s], dst, x, y);
-                else tma_load_2d_pair(mapB, fb, dst, x, y);
-              }
-            }
-            ++issued;
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
+          const uint32_t s = issued % kNS;
+          const uint32_t ph = (issued / kNS) & 1u;
+          if (!wait_bar(&empty_bar[s], ph ^ 1u, ctl, kPark)) {
+            ok = false;
+            break;
           }
+          uint8_t* a_s = smem + s * kSBytes;
+          uint8_t* b_s = a_s + kATileBytes;
+          if (kLocalCopies) mbar_arrive_expect_tx(&full_bar[s], kSBytes);
+          else if (leader) mbar_arrive_expect_tx(&full_bar[s], kSBytes * kCtas);
+          const uint32_t fb = kLocalCopies ? 0u : mapa_shared(&full_bar[s], 0);
+          const int k0 = kb * kBKe;
+#pragma unroll
+          for (int sl = 0; sl < (A_MN ? kBM / kMNe : 1); ++sl) {
+            void* dst = a_s + sl * kSlabBytes;
+            const int x = A_MN ? m0 + sl * kMNe : k0, y = A_MN ? k0 : m0;
+            if (kLocalCopies) tma_load_2d(&tmA, &full_bar[s], dst, x, y);
+            else tma_load_2d_pair(&tmA, fb, dst, x, y);
+          }
+#pragma unroll
+          for (int h = 0; h < kHalves; ++h) {
+            const int nh = n0 + h * kBN;  // this CTA's B rows of half h
+#pragma unroll
+            for (int sl = 0; sl < (B_MN ? kBRows / kMNe : 1); ++sl) {
+              void* dst = b_s + h * kBBytes + sl * kSlabBytes;
+              const int x = B_MN ? nh + sl * kMNe : k0, y = B_MN ? k0 : nh;
+              if (kLocalCopies) tma_load_2d(&tmB, &full_bar[s], dst, x, y);
+              else tma_load_2d_pair(&tmB, fb, dst, x, y);
+            }
+          }
+          ++issued;
         }
       }
       *issued_slot = issued;
@@ -466,63 +413,58 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       uint32_t consumed = 0, local = 0;
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += units, ++local) {
+        const uint32_t buf = local % kAccBufs;
+        const uint32_t aph = (local / kAccBufs) & 1u;
+        if (!wait_bar(&tempty_bar[buf], aph ^ 1u, ctl, kPark)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * kBN;
         const UnitRange ur = unit_range(t, p);
-        for (int part = 0; part < kParts && ok; ++part) {
-          // DUAL: each unit fills accumulator 0 (teacher) and then 1 (student)
-          const uint32_t buf = EPI == EPI_DUAL ? static_cast<uint32_t>(part) : local % kAccBufs;
-          const uint32_t aph = (EPI == EPI_DUAL ? local : local / kAccBufs) & 1u;
-          if (!wait_bar(&tempty_bar[buf], aph ^ 1u, ctl, kPark)) {
+        for (int kb = ur.kb0; kb < ur.kb1; ++kb) {
+          const uint32_t s = consumed % kNS;
+          const uint32_t ph = (consumed / kNS) & 1u;
+          const bool got = XF ? wait_bar(&ready_bar[s], ph, ctl, kPark)
+                              : wait_bar(&full_bar[s], ph, ctl, kPark);
+          if (!got) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + buf * kBN;
-          int kbb, kbe;
-          part_kb(ur, part, kbb, kbe);
-          for (int kb = kbb; kb < kbe; ++kb) {
-            const uint32_t s = consumed % kNS;
-            const uint32_t ph = (consumed / kNS) & 1u;
-            const bool got = XF ? wait_bar(&ready_bar[s], ph, ctl, kPark)
-                                : wait_bar(&full_bar[s], ph, ctl, kPark);
-            if (!got) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + s * kSBytes);
-            const uint32_t b_addr = a_addr + kATileBytes;
+          const uint32_t a_addr = smem_u32(smem + s * kSBytes);
+          const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
-            for (int j = 0; j < kKSteps; ++j) {
-              const uint64_t ad = A_MN ? sdesc_sw128(a_addr + j * (kUmmaK / 8) * 1024,
+          for (int j = 0; j < kKSteps; ++j) {
+            const uint64_t ad = A_MN ? sdesc_sw128(a_addr + j * (kUmmaK / 8) * 1024,
+                                                   kSlabBytes, 1024)
+                                     : sdesc_sw128(a_addr + j * 32, 16, 1024);
+            const uint32_t acc = (kb != ur.kb0 || j != 0) ? 1u : 0u;
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+              const uint32_t bh = b_addr + h * kBBytes;
+              const uint64_t bd = B_MN ? sdesc_sw128(bh + j * (kUmmaK / 8) * 1024,
                                                      kSlabBytes, 1024)
-                                       : sdesc_sw128(a_addr + j * 32, 16, 1024);
-              const uint32_t acc = (kb != kbb || j != 0) ? 1u : 0u;
-#pragma unroll
-              for (int h = 0; h < kHalves; ++h) {
-                const uint32_t bh = b_addr + h * kBBytes;
-                const uint64_t bd = B_MN ? sdesc_sw128(bh + j * (kUmmaK / 8) * 1024,
-                                                       kSlabBytes, 1024)
-                                         : sdesc_sw128(bh + j * 32, 16, 1024);
-                const uint32_t dh = d_tmem + h * kBN;
-                if (PAIR) {
-                  if (kEB == 2) umma_f16_pair(dh, ad, bd, kIdesc, acc);
-                  else umma_tf32_pair(dh, ad, bd, kIdesc, acc);
-                } else {
-                  if (kEB == 2) umma_f16(dh, ad, bd, kIdesc, acc);
-                  else umma_tf32(dh, ad, bd, kIdesc, acc);
-                }
+                                       : sdesc_sw128(bh + j * 32, 16, 1024);
+              const uint32_t dh = d_tmem + h * kBN;
+              if (PAIR) {
+                if (kEB == 2) umma_f16_pair(dh, ad, bd, kIdesc, acc);
+                else umma_tf32_pair(dh, ad, bd, kIdesc, acc);
+              } else {
+                if (kEB == 2) umma_f16(dh, ad, bd, kIdesc, acc);
+                else umma_tf32(dh, ad, bd, kIdesc, acc);
               }
             }
-            // frees the smem stage (in both CTAs of a pair) when these MMAs finish
-            if (PAIR) umma_commit_pair(&empty_bar[s], 0x3);
-            else umma_commit(&empty_bar[s]);
-            ++consumed;
           }
-          if (!ok) break;
-          // accumulator ready for the epilogue(s)
-          if (PAIR) umma_commit_pair(&tfull_bar[buf], 0x3);
-          else umma_commit(&tfull_bar[buf]);
+          // frees the smem stage (in both CTAs of a pair) when these MMAs finish
+          if (PAIR) umma_commit_pair(&empty_bar[s], 0x3);
+          else umma_commit(&empty_bar[s]);
+          ++consumed;
         }
+        if (!ok) break;
+        // accumulator ready for the epilogue(s)
+        if (PAIR) umma_commit_pair(&tfull_bar[buf], 0x3);
+        else umma_commit(&tfull_bar[buf]);
       }
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is released.
@@ -632,10 +574,10 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       }
     };
     // Stage v * scale - shift (32 values of this thread's row) and store the
-    // warp's box through `map` at output column x, output-map row y (rows past
-    // the map's extent are not written).
+    // warp's box at output column x, output-map row y (rows past the map's
+    // extent are not written).
     auto store_box = [&](const uint32_t(&v)[32], float scale, float shift, int x, int y,
-                         bool fp32_out, bool reduce, bool issue, const CUtensorMap* map) {
+                         bool fp32_out, bool reduce, bool issue) {
       uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
       ++nbox;
       if (lane == 0) bulk_wait_read_1();  // the store that last used sb has read it
@@ -665,146 +607,16 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       if (lane == 0 && issue) {
         // outputs are streamed, never re-read by this kernel: evict them from
         // L2 first so the operand tiles that other tiles share stay resident
-        if (reduce) tma_reduce_add_2d_hint(map, sb, x, y, out_policy);
-        else tma_store_2d_hint(map, sb, x, y, out_policy);
+        if (reduce) tma_reduce_add_2d_hint(&tmC, sb, x, y, out_policy);
+        else tma_store_2d_hint(&tmC, sb, x, y, out_policy);
         bulk_commit();
       }
     };
     constexpr bool kElemF32 = sizeof(Elem) == 4;
-    // EPI_DUAL, one unit (output tile tm, tn; the unit's ordinal `ord` among
-    // this CTA's units); false when the CTA aborted.
-    auto dual_unit = [&](int tm, int tn, uint32_t ord) -> bool {
-      const int row0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM + warp * 32;
-      const int grow = row0 + lane;
-      const bool rv = grow < p.rows_valid;
-      const bool warp_rows = row0 < p.rows_valid;
-      const int col0 = tn * kBN;
-      const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
-      const float s2 = rscale * kLog2e;
-      const uint32_t aph = ord & 1u;  // each accumulator completes once per unit
-      const uint32_t tb0 = tmem_base + lane_base;         // teacher: columns 0-255
-      const uint32_t tb1 = tmem_base + lane_base + kBN;   // student: columns 256-511
-      // This thread's row of the CTA's scratch: the float4 (slab c, chunk j) of
-      // CTA row r sits at (8 c + j) * kBM + r, so that a warp's 32 lanes write
-      // and read 512 contiguous bytes.  Each thread reads back only what it
-      // wrote itself; the values stay in L2 between the two halves.
-      float4* scr = p.tscr + static_cast<int64_t>(blockIdx.x) * (kDualScratchBytes / 16) +
-                    warp * 32 + lane;
-      // Row maximum over the tile of accumulator `tb` (base-2 units).
-      auto tile_max = [&](uint32_t tb) {
-        float m = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(tb + c * 32, v);
-          tmem_ld_wait();
-          const int nvalid = p.cols_valid - (col0 + c * 32);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            m = fmaxf(m, i < nvalid ? __uint_as_float(v[i]) * s2 : -INFINITY);
-        }
-        return m;
-      };
-
-      // ---- teacher half: statistics, t~ - max kept in the scratch (fp32) and
-      // optionally stored through tmF; the columns are released after the last
-      // TMEM read so that the next unit's teacher MMAs can start
-      if (!wait_bar(&tfull_bar[0], aph, ctl, kPark)) return false;
-      __syncwarp();
-      tc_fence_after();
-      const float mt = tile_max(tb0);
-      const float tshift = mt > -INFINITY ? mt * kLn2f : 0.f;  // natural units
-      float zt = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld32(tb0 + c * 32, v);
-        tmem_ld_wait();
-        if (c == kBN / 32 - 1) release(0);
-        const int cb = col0 + c * 32;
-        const int nvalid = p.cols_valid - cb;
-        if (nvalid <= 0) continue;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          zt += i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mt)) : 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          __stcg(scr + (c * 8 + j) * kBM,
-                 make_float4(fmaf(__uint_as_float(v[4 * j]), rscale, -tshift),
-                             fmaf(__uint_as_float(v[4 * j + 1]), rscale, -tshift),
-                             fmaf(__uint_as_float(v[4 * j + 2]), rscale, -tshift),
-                             fmaf(__uint_as_float(v[4 * j + 3]), rscale, -tshift)));
-        if (p.store_t)
-          store_box(v, rscale, tshift, cb, row0, p.t_f32 != 0, false, warp_rows, &tmF);
-      }
-      if (rv) p.tpartials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mt, zt, 0.f, 0.f);
-
-      // ---- student half: statistics and the tile sums
-      //   A = sum 2^(t - mt) (t~ - s~),  U = sum 2^(s - ms) (s~ - t~)
-      // from the fp32 accumulator and the fp32 teacher values (loaded one slab
-      // ahead, so that their latency overlaps the previous slab's work)
-      if (!wait_bar(&tfull_bar[1], aph, ctl, kPark)) return false;
-      __syncwarp();
-      tc_fence_after();
-      auto load_t = [&](int c, float(&tv)[32]) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 t4 = __ldcg(scr + (c * 8 + j) * kBM);
-          tv[4 * j] = t4.x;
-          tv[4 * j + 1] = t4.y;
-          tv[4 * j + 2] = t4.z;
-          tv[4 * j + 3] = t4.w;
-        }
-      };
-      float tcur[32];
-      load_t(0, tcur);
-      const float ms = tile_max(tb1);
-      const float sshift = ms > -INFINITY ? ms * kLn2f : 0.f;
-      float se = 0.f, A = 0.f, U = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld32(tb1 + c * 32, v);
-        tmem_ld_wait();
-        if (c == kBN / 32 - 1) release(1);
-        const int cb = col0 + c * 32;
-        const int nvalid = p.cols_valid - cb;
-        if (nvalid <= 0) continue;
-        float tnxt[32];
-        const bool more = c + 1 < kBN / 32 && nvalid > 32;
-        if (more) load_t(c + 1, tnxt);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i < nvalid) {
-            const float x = __uint_as_float(v[i]);
-            const float e = ex2_approx(fmaf(x, s2, -ms));
-            const float d = (tcur[i] + tshift) - x * rscale;  // t~ - s~
-            se += e;
-            A = fmaf(ex2_approx(tcur[i] * kLog2e), d, A);
-            U = fmaf(e, -d, U);
-          }
-        }
-        if (p.store == STORE_SHIFTED)
-          store_box(v, rscale, sshift, cb, row0, kElemF32, false, warp_rows, &tmC);
-        if (more) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) tcur[i] = tnxt[i];
-        }
-      }
-      if (rv) p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(ms, se, A, U);
-      return true;
-    };
     for (int t = unit; t < total_tiles; t += units, ++local) {
       const UnitRange ur = unit_range(t, p);
       int tm, tn;
       tile_coords(ur.tile, p, tm, tn);
-      if (EPI == EPI_DUAL) {
-        if (!dual_unit(tm, tn, local)) break;
-        continue;
-      }
       const uint32_t buf = local % kAccBufs;
       const uint32_t aph = (local / kAccBufs) & 1u;
       if (!wait_bar(&tfull_bar[buf], aph, ctl, kPark)) break;
@@ -835,6 +647,32 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
           gi = lo;
           gcol = gi < p.ktop ? __ldg(ri + gi) : 0x7fffffff;
         }
+        // Teacher-hidden student pass (tbuf given): the teacher's stored tile
+        // t~ - mt gives, per column, w = 2^((t~ - mt) log2 e) and t~ - s~; the
+        // tile's sums A = sum w (t~ - s~) and U = sum 2^(x - max) (s~ - t~) are
+        // formed in pass 2 from fp32 values.  The teacher values of a 32-column
+        // slab are loaded one slab ahead (slab 0 before pass 1) so that their
+        // latency overlaps the work on the previous slab.
+        const bool hid = p.tbuf != nullptr && rv;
+        const float* trow = hid ? p.tbuf + static_cast<int64_t>(grow) * p.tld : nullptr;
+        auto load_t = [&](int cb, float(&tv)[32]) {
+          const int nv = p.cols_valid - cb;
+          if (nv >= 32) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 t4 = __ldg(reinterpret_cast<const float4*>(trow + cb) + j);
+              tv[4 * j] = t4.x;
+              tv[4 * j + 1] = t4.y;
+              tv[4 * j + 2] = t4.z;
+              tv[4 * j + 3] = t4.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) tv[i] = i < nv ? __ldg(trow + cb + i) : 0.f;
+          }
+        };
+        float tcur[32];
+        if (hid) load_t(col0, tcur);
         // Pass 1: the row's maximum over this tile (base-2 units) and the
         // cached entries' cross term, from the fp32 accumulator.
 #pragma unroll 1
@@ -863,6 +701,10 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
         // 0, where the stored value's rounding error vanishes; readers add the
         // maximum back from the tile statistics.  STORE_EXP stores the
         // exponentials 2^(x - max) in (0, 1].
+        const float mt = hid ? __ldg(&p.tpart[static_cast<int64_t>(grow) * p.tiles_n + tn].x) *
+                                   kLn2f
+                             : 0.f;
+        float A = 0.f, U = 0.f;
         const float shift = (p.partials != nullptr && mx > -INFINITY) ? mx * kLn2f : 0.f;
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
@@ -880,17 +722,35 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
             e[i] = i < nvalid ? ex2_approx(fmaf(__uint_as_float(v[i]), s2, -mx)) : 0.f;
             se += e[i];
           }
+          if (hid) {
+            float tnxt[32];
+            const bool more = c + 1 < kBN / 32 && nvalid > 32;
+            if (more) load_t(cb + 32, tnxt);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < nvalid) {
+                const float d = (tcur[i] + mt) - __uint_as_float(v[i]) * rscale;  // t~ - s~
+                A = fmaf(ex2_approx(tcur[i] * kLog2e), d, A);
+                U = fmaf(e[i], -d, U);
+              }
+            }
+            if (more) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) tcur[i] = tnxt[i];
+            }
+          }
           if (p.store == STORE_SHIFTED) {
-            store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows, &tmC);
+            store_box(v, rscale, shift, cb, row0, p.out_f32 != 0, false, warp_rows);
           } else if (p.store == STORE_EXP) {
             uint32_t eb[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) eb[i] = __float_as_uint(e[i]);
-            store_box(eb, 1.f, 0.f, cb, row0, false, false, warp_rows, &tmC);
+            store_box(eb, 1.f, 0.f, cb, row0, false, false, warp_rows);
           }
         }
         if (rv && p.partials != nullptr)
-          p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] = make_float4(mx, se, cross, 0.f);
+          p.partials[static_cast<int64_t>(grow) * p.tiles_n + tn] =
+              p.tbuf != nullptr ? make_float4(mx, se, A, U) : make_float4(mx, se, cross, 0.f);
       } else if (EPI == EPI_DLOGITS) {
         float coef = 0.f, cm = 0.f, l2 = 0.f;
         const float rscale = (p.T_row != nullptr && rv) ? 1.f / p.T_row[grow] : p.scale;
@@ -942,7 +802,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(round_tf32_dev(__uint_as_float(v[i])));
           }
-          store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows, &tmC);
+          store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows);
         }
       } else {
 #pragma unroll 1
@@ -955,10 +815,9 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
           const int cb = col0 + c * 32;
           if (cb >= p.cols_valid) continue;
           if (EPI == EPI_STORE)
-            store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows, &tmC);
+            store_box(v, 1.f, 0.f, cb, row0, kElemF32, false, warp_rows);
           else  // EPI_ACCUM, fp32 out; K-part ks writes its own block of output rows
-            store_box(v, 1.f, 0.f, cb, row0 + ur.ks * p.split_rows, true, p.beta != 0, warp_rows,
-                    &tmC);
+            store_box(v, 1.f, 0.f, cb, row0 + ur.ks * p.split_rows, true, p.beta != 0, warp_rows);
         }
       }
     }

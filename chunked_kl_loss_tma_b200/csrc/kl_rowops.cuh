@@ -493,12 +493,11 @@ __global__ void hidden_sums_kernel(const float4* __restrict__ part_s,
 // Full-vocabulary mode, dS in place over the student buffer (one CTA per row):
 //   dS = c [(1 - beta)(p_s - p_t) + beta p_s (u - u_bar)],  u = s~ - t~,
 // c = g / (n T) (0 on masked rows), with p_s from the stored s~ - ms (element
-// type of H) and p_t from the stored t~ - mt (TElem: the element type, or fp32
-// where the reverse term needs s~ - t~ to fp32 accuracy), the tile maxima
-// (base 2) from the logits pass's statistics, the row lse's and u_bar per row.
-// Columns from V to the row's padded end are written as 0.
-template <typename Elem, typename TElem>
-__global__ void dlogits_full_kernel(Elem* __restrict__ S, const TElem* __restrict__ Tt, int64_t ld,
+// type of H), p_t from the stored t~ - mt (fp32), the tile maxima (base 2)
+// from the two passes' statistics, the row lse's and u_bar per row.  Columns
+// from V to the row's padded end are written as 0.
+template <typename Elem>
+__global__ void dlogits_full_kernel(Elem* __restrict__ S, const float* __restrict__ Tt, int64_t ld,
                                     int V, const float* __restrict__ lse_s,
                                     const float* __restrict__ lse_t,
                                     const float* __restrict__ ubar,
@@ -509,7 +508,7 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const TElem* __restric
                                     const float4* __restrict__ part_t, int tiles_n) {
   const int row = blockIdx.x;
   Elem* srow = S + static_cast<int64_t>(row) * ld;
-  const TElem* trow = Tt + static_cast<int64_t>(row) * ld;
+  const float* trow = Tt + static_cast<int64_t>(row) * ld;
   const float coef = grad_coef(mask, row, sc, g_dev, g_host, invT, T_row);
   const float ls2 = lse_s[row] * kLog2e, lt2 = lse_t[row] * kLog2e;
   const float cf = coef * (1.f - beta), cr = coef * beta;
@@ -518,7 +517,7 @@ __global__ void dlogits_full_kernel(Elem* __restrict__ S, const TElem* __restric
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float fs[8], ft[8];
     load8<Elem>(srow + v * 8, fs);
-    load8<TElem>(trow + v * 8, ft);
+    load8<float>(trow + v * 8, ft);
     // 8 | 256: the vector lies in one tile
     const float ms2 = part_s[static_cast<int64_t>(row) * tiles_n + (v >> 5)].x;
     const float mt2 = part_t[static_cast<int64_t>(row) * tiles_n + (v >> 5)].x;

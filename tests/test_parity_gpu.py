@@ -323,14 +323,15 @@ def test_launch_counter_and_profile():
     names = {p["name"] for p in L.kl_profile_end()}
     assert {"gemm_logits_stats", "xf_patch", "xf_scales", "gemm_dH", "gemm_dW"} <= names
     assert "dlogits_topk" not in names
-    # teacher-hidden mode: both logit tiles of a chunk in one launch per chunk
+    # teacher-hidden mode: the teacher pass, then the student pass, per chunk
     h = _small_hidden(seed=26)
     L.kl_profile_begin()
     ops.kl_fwd_bwd(h.H, h.W, **_kw(h, chunk=128))
     prof = {p["name"]: p for p in L.kl_profile_end()}
-    assert {"gemm_logits_dual", "hidden_sums", "dlogits_full", "gemm_dH", "gemm_dW"} <= set(prof)
-    assert "gemm_logits_stats" not in prof
-    assert prof["gemm_logits_dual"]["launches"] == -(-h.N // 128)
+    assert {"gemm_teacher_logits", "gemm_logits_stats", "hidden_sums", "dlogits_full",
+            "gemm_dH", "gemm_dW"} <= set(prof)
+    chunks = -(-h.N // 128)
+    assert prof["gemm_teacher_logits"]["launches"] == prof["gemm_logits_stats"]["launches"] == chunks
 
 
 def test_bitwise_deterministic_across_calls():
