@@ -8,8 +8,9 @@ same mean.  Then the ranks' head gradients dW and their loss shares are summed
 (all-reduce), or dW is reduce-scattered into row shards, as a sharded
 optimizer keeps them.  dH stays with the rank that owns the tokens.
 
-NCCL reduces device tensors in place; another backend (gloo) stages them
-through host memory."""
+NCCL reduces device tensors in place, also in a group of one rank (so a one-GPU
+run takes the multi-GPU path); another backend (gloo) stages them through host
+memory, and a group of one gloo rank exchanges nothing."""
 from __future__ import annotations
 
 import torch
@@ -60,7 +61,7 @@ def dW_shard_rows(V: int, world: int, rank: int):
 def sum_over_ranks(t: torch.Tensor, group=None, async_op: bool = False):
     """In-place sum of `t` over the ranks.  With NCCL and async_op, returns the
     work handle to wait on; otherwise the sum is complete on return."""
-    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+    if not dist.is_initialized() or (dist.get_world_size(group) == 1 and not _nccl(group)):
         return None
     if _nccl(group):
         return dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
@@ -75,7 +76,7 @@ def reduce_scatter_rows(t: torch.Tensor, group=None) -> torch.Tensor:
     (dW_shard_rows); a copy padded to the block size."""
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     rank = dist.get_rank(group) if dist.is_initialized() else 0
-    if world == 1:
+    if world == 1 and not _nccl(group):
         return t
     V = t.shape[0]
     per = -(-V // world)

@@ -156,18 +156,20 @@ class ShardPass:
 
 class TorchComm:
     """The pass's collectives over a torch.distributed process group: NCCL on
-    device tensors; with another backend (gloo) device tensors go through host
-    copies and the reductions run synchronously."""
+    device tensors (issued even for a group of one rank, so that a one-GPU run
+    takes the same path as a multi-GPU one); with another backend (gloo) device
+    tensors go through host copies and the reductions run synchronously; with
+    no process group, one rank and no collectives."""
 
     def __init__(self, group=None):
         self.group = group
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
-        self.nccl = self.world > 1 and dist.get_backend(group) == "nccl"
+        self.nccl = dist.is_initialized() and dist.get_backend(group) == "nccl"
 
     def all_gather_rows(self, t):
         """[rows, k] from every rank -> [world * rows, k], rank-major."""
-        if self.world == 1:
+        if self.world == 1 and not self.nccl:
             return t
         if self.nccl:
             out = torch.empty((self.world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype,
@@ -181,7 +183,7 @@ class TorchComm:
 
     def all_reduce_sum(self, t, async_op=False):
         """In-place sum over ranks; a handle to wait on when async_op and NCCL."""
-        if self.world == 1:
+        if self.world == 1 and not self.nccl:
             return None
         if self.nccl:
             return dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group, async_op=async_op)
