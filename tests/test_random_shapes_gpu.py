@@ -9,6 +9,10 @@ probabilities, a reverse-KL weight in the teacher-hidden mode, and the entry:
 the fused pass (with or without dS formed inside the dH contraction) or kl_fwd
 followed by kl_bwd (with or without the kept last chunk).
 
+A second set of seeds runs the vocabulary-parallel form (`vocab_parallel.emulate`,
+the head cut into 2 to 4 shards at random rows) against the oracle on the
+whole problem.
+
 Tolerances as in the other parity tests: loss relative error <= 1e-3 (plus 1e-6
 absolute, for losses that are 0), gradients max-abs error <= 2e-2 * max|oracle
 gradient|."""
@@ -100,4 +104,70 @@ def test_random_problem_matches_oracle(seed):
     for name, got in (("dH", dH), ("dW", dW)):
         r = ref[name]
         err = np.max(np.abs(got.double().cpu().numpy() - r))
+        assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
+
+
+VP_CASES = 16
+
+
+def _draw_vp(seed):
+    """A random problem for the vocabulary-parallel form: as _draw, with the head
+    cut into P = 2..4 shards at random rows (boundaries inside tiles, shards of
+    a few rows among them)."""
+    rng = np.random.default_rng(7000 + seed)
+    mode = "hidden" if rng.random() < 0.45 else "topk"
+    dtype = torch.float32 if rng.random() < 0.2 else torch.bfloat16
+    N = int(rng.integers(1, 400))
+    d = 8 * int(rng.integers(1, 40))
+    P = int(rng.integers(2, 5))
+    V = int(rng.integers(P + 1, 6000))
+    cuts = np.sort(rng.choice(np.arange(1, V), size=P - 1, replace=False))
+    bounds = [0] + [int(c) for c in cuts] + [V]
+    shards = [(bounds[i], bounds[i + 1]) for i in range(P)]
+    K = int(rng.integers(1, min(V, 64) + 1))
+    d_t = 8 * int(rng.integers(1, 24))
+    T = float(rng.uniform(0.5, 3.0))
+    Tr = torch.from_numpy(rng.uniform(0.5, 3.0, size=N).astype(np.float32)) \
+        if rng.random() < 0.3 else None
+    chunk = int(rng.choice([0, 64, 200]))
+    beta = float(rng.choice([0.0, 0.4, 1.0])) if mode == "hidden" else 0.0
+    fuse = bool(mode == "topk" and dtype == torch.bfloat16 and rng.random() < 0.4)
+    g = float(rng.uniform(0.3, 2.0))
+    w_std = float(rng.uniform(0.03, 0.3))
+    if mode == "topk":
+        w = wl.make_topk(f"vp{seed}", N=N, d=d, V=V, K=K, d_t=d_t,
+                         T=Tr if Tr is not None else T, dtype=dtype, w_std=w_std,
+                         tw_std=float(rng.uniform(0.05, 0.3)), seed=8000 + seed,
+                         partial_mass=rng.random() < 0.6)
+    else:
+        w = wl.make_hidden(f"vph{seed}", N=N, d=d, d_t=d_t, V=V,
+                           T=Tr if Tr is not None else T, dtype=dtype, w_std=w_std,
+                           tw_std=float(rng.uniform(0.05, 0.3)), seed=8000 + seed)
+    if rng.random() < 0.5:
+        w.mask = torch.from_numpy((rng.random(N) > 0.25).astype(np.uint8))
+    return w.to("cuda"), dict(shards=shards, chunk=chunk, beta=beta, fuse=fuse, g=g)
+
+
+@pytest.mark.parametrize("seed", range(VP_CASES))
+def test_random_vocabulary_shards_match_oracle(seed):
+    from chunked_kl_loss_tma_b200 import vocab_parallel as vp
+
+    w, o = _draw_vp(seed)
+    kw = _kw(w, o)
+    Wt = kw.pop("Wt", None)
+    out = vp.emulate(w.H, w.W, len(o["shards"]), shards=o["shards"], grad_loss=o["g"], Wt=Wt,
+                     fuse_dlogits=o["fuse"], **kw)
+    assert all(ops.status(ws) == 0 for ws in out["workspaces"])
+    args = dict(T=w.T, mask=w.mask, mode=w.mode, grad_loss=o["g"], reverse_weight=o["beta"])
+    if w.mode == "topk":
+        args.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        args.update(Ht=w.Ht, Wt=w.Wt)
+    ref = oracle.kl_loss(w.H, w.W, **args)
+    case = f"vp seed {seed}: N={w.N} d={w.d} V={w.V} {w.mode} {w.dtype} {o}"
+    assert abs(out["loss"].item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-6, \
+        (case, out["loss"].item(), ref["loss"])
+    for name in ("dH", "dW"):
+        r = ref[name]
+        err = np.max(np.abs(out[name].double().cpu().numpy() - r))
         assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
