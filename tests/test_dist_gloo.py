@@ -104,18 +104,20 @@ def _reduce_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_sum_and_reduce_scatter_helpers():
+@pytest.mark.parametrize("world", [1, 2])
+def test_sum_and_reduce_scatter_helpers(world):
     """sum_over_ranks and reduce_scatter_rows (the head-gradient reductions of
-    the token data-parallel form) over gloo, against the plain sums."""
+    the token data-parallel form) over gloo, against the plain sums; a group of
+    one gloo rank leaves the tensor as it is."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_reduce_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_reduce_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = sorted(q.get(timeout=120) for _ in range(2))
+    res = sorted(q.get(timeout=120) for _ in range(world))
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(r[1] and r[2] for r in res), res
-    assert [r[3] for r in res] == [(0, 6), (6, 11)]
+    assert [r[3] for r in res] == ([(0, 11)] if world == 1 else [(0, 6), (6, 11)])
