@@ -175,3 +175,38 @@ def test_fuse_dlogits_flag_rules(lib):
     assert L.kl_fwd(p, dummy, base, dummy, dummy, None, None, None) == 10  # KL_ERR_ARG
     assert L.kl_bwd(p, dummy, base, dummy, None, dummy, dummy, dummy, 0, None) == 10
     assert L.kl_fwd_noalloc(p, dummy, dummy, dummy, None, None) == 10
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """The header compiles as strict C99, the library links from C, and a C
+    caller gets the answers the Python binding gets (tests/abi_c_caller.c)."""
+    import ctypes
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    here = os.path.dirname(__file__)
+    libdir = os.path.dirname(B.OUT)
+    exe = str(tmp_path / "abi_c_caller")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.dirname(HEADER), os.path.join(here, "abi_c_caller.c"),
+                    "-L", libdir, "-lchunkedkl", "-Wl,-rpath," + libdir, "-o", exe],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    assert int(got["sizeof_problem"]) == ctypes.sizeof(L.KLProblem)
+    for e in (L.KL_ENTRY_FWD, L.KL_ENTRY_BWD, L.KL_ENTRY_FWD_BWD):
+        assert int(got[f"ws_topk_{e}"]) == L.kl_workspace_bytes(_problem(), e)
+    hidden = _problem(teacher=1, K=0, d_t=4096, N=8192, T=2.0)
+    assert int(got["ws_hidden"]) == L.kl_workspace_bytes(hidden, L.KL_ENTRY_FWD_BWD)
+    code = {name: c for c, name in L.STATUS.items()}
+    assert int(got["ws_bad_T"]) == 0
+    assert int(got["fwd_bwd_bad_T"]) == code["KL_ERR_ARG"]
+    assert int(got["fwd_bwd_bad_d"]) == code["KL_ERR_ALIGN"]
+    assert int(got["fwd_null_inputs"]) == code["KL_ERR_NULL"]
+    assert int(got["fwd_bwd_null"]) == code["KL_ERR_NULL"]
+    assert got["status_string_align"] == L.kl_status_string(code["KL_ERR_ALIGN"])
+    assert int(got["noalloc_scratch"]) == L.KL_NOALLOC_SCRATCH_BYTES
+
