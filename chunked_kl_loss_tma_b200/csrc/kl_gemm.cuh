@@ -575,9 +575,14 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     };
     // Stage v * scale - shift (32 values of this thread's row) and store the
     // warp's box at output column x, output-map row y (rows past the map's
-    // extent are not written).
+    // extent are not written).  issue is false (uniformly over the warp) when
+    // all of the warp's rows lie past the output's extent: then nothing is
+    // staged either.  Each staged box commits exactly one bulk group, which is
+    // what lets the wait below (at most one group still reading) prove that
+    // the store which last used this buffer, two boxes back, has read it.
     auto store_box = [&](const uint32_t(&v)[32], float scale, float shift, int x, int y,
                          bool fp32_out, bool reduce, bool issue) {
+      if (!issue) return;
       uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
       ++nbox;
       if (lane == 0) bulk_wait_read_1();  // the store that last used sb has read it
@@ -604,7 +609,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0 && issue) {
+      if (lane == 0) {
         // outputs are streamed, never re-read by this kernel: evict them from
         // L2 first so the operand tiles that other tiles share stay resident
         if (reduce) tma_reduce_add_2d_hint(&tmC, sb, x, y, out_policy);

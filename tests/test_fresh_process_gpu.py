@@ -1,0 +1,57 @@
+"""The first call in a fresh process against the next one.  Every reduction
+here has a fixed order, so a call's results do not depend on what ran before
+it: the first call (cold caches and TLBs, freshly mapped output buffers, so
+TMA stores run slowly) must equal the second bit for bit.  The case is chosen
+so that an epilogue warp alternates between units whose rows exist and units
+whose rows lie past the output (dW: V = 1500 is not a multiple of 256), with
+short units (two K-blocks per dW unit) and 8192-wide rows.  A staging buffer
+reused while a slow TMA store still read it once corrupted one 32 x 32 box of
+dW on the first call in about half of the processes."""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+PROCESSES = 4
+
+
+def _worker(q):
+    import numpy as np
+
+    from chunked_kl_loss_tma_b200 import ops
+    from chunked_kl_loss_tma_b200 import workloads as wl
+
+    try:
+        torch.cuda.set_device(0)
+        w = wl.make_topk("fresh", N=300, d=8192, V=1500, K=32, d_t=64, T=1.5,
+                         dtype=torch.bfloat16, w_std=0.02, tw_std=0.05, seed=41).to("cuda")
+        kw = dict(T=w.T, chunk_tokens=128, topk_idx=w.topk_idx, topk_logit=w.topk_logit,
+                  teacher_lse=w.teacher_lse)
+        outs = [ops.kl_fwd_bwd(w.H, w.W, **kw) for _ in range(2)]
+        torch.cuda.synchronize()
+        a, b = outs
+        diff = float((a["dW"] - b["dW"]).abs().max().item())
+        q.put(dict(status=[ops.status(o["workspace"]) for o in outs],
+                   same=bool(torch.equal(a["loss"], b["loss"]) and
+                             torch.equal(a["dH"], b["dH"]) and
+                             torch.equal(a["dW"], b["dW"])),
+                   dW_diff=diff, dW_scale=float(np.abs(b["dW"].cpu().numpy()).max())))
+    except Exception as e:  # report instead of leaving the parent waiting
+        q.put(dict(error=repr(e)))
+
+
+def test_first_call_equals_second_in_fresh_processes():
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    results = []
+    for _ in range(PROCESSES):
+        q = ctx.Queue()
+        p = ctx.Process(target=_worker, args=(q,))
+        p.start()
+        results.append(q.get(timeout=300))
+        p.join(timeout=120)
+    for r in results:
+        assert "error" not in r, r
+        assert r["status"] == [0, 0], r
+        assert r["same"], r

@@ -425,6 +425,34 @@ def test_max_cache_size_K1024():
     _check_grad(out["dW"], ref["dW"], "dW")
 
 
+@pytest.mark.parametrize("mode,d,d_t", [("topk", 8192, 64), ("hidden", 8192, 1024),
+                                         ("hidden", 512, 8192)])
+def test_wide_heads(mode, d, d_t):
+    """Hidden widths well above the bench's 3072 (128 K-blocks per logits tile,
+    8192-wide dH rows and dW columns), through the fused call and the split pair
+    with the last chunk kept, with a ragged last chunk."""
+    if mode == "topk":
+        w = wl.make_topk("wide", N=300, d=d, V=1500, K=32, d_t=d_t, T=1.5,
+                         dtype=torch.bfloat16, w_std=0.02, tw_std=0.05, seed=41).to("cuda")
+    else:
+        w = wl.make_hidden("wideh", N=300, d=d, d_t=d_t, V=1500, T=1.5, dtype=torch.bfloat16,
+                           w_std=0.02, tw_std=0.02, seed=42).to("cuda")
+    ref = _oracle(w)
+    kw = _kw(w, chunk=128)
+    out = ops.kl_fwd_bwd(w.H, w.W, **kw)
+    assert ops.status(out["workspace"]) == 0
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+    f = ops.kl_fwd(w.H, w.W, keep_last_chunk=True, **kw)
+    b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"], workspace=f["workspace"],
+                   keep_last_chunk=True, **kw)
+    assert ops.status(f["workspace"]) == 0
+    _check_loss(f["loss"].item(), ref["loss"])
+    _check_grad(b["dH"], ref["dH"], "dH (split)")
+    _check_grad(b["dW"], ref["dW"], "dW (split)")
+
+
 @pytest.mark.parametrize("mode", ["topk", "hidden"])
 def test_vocabulary_smaller_than_one_tile(mode):
     if mode == "topk":
