@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 PROCESSES = 4
 
 
-def _worker(q):
+def _worker(case, q):
     import numpy as np
 
     from chunked_kl_loss_tma_b200 import ops
@@ -23,10 +23,16 @@ def _worker(q):
 
     try:
         torch.cuda.set_device(0)
-        w = wl.make_topk("fresh", N=300, d=8192, V=1500, K=32, d_t=64, T=1.5,
-                         dtype=torch.bfloat16, w_std=0.02, tw_std=0.05, seed=41).to("cuda")
-        kw = dict(T=w.T, chunk_tokens=128, topk_idx=w.topk_idx, topk_logit=w.topk_logit,
-                  teacher_lse=w.teacher_lse)
+        if case == "hidden":
+            w = wl.make_hidden("fresh_h", N=300, d=8192, d_t=1024, V=1500, T=1.7,
+                               dtype=torch.bfloat16, w_std=0.02, tw_std=0.02, seed=2).to("cuda")
+            kw = dict(T=w.T, chunk_tokens=128, Ht=w.Ht, Wt=w.Wt)
+        else:
+            w = wl.make_topk("fresh", N=300, d=8192 if case == "topk" else 4096, V=1500, K=32,
+                             d_t=64, T=1.5, dtype=torch.bfloat16, w_std=0.02, tw_std=0.05,
+                             seed=41).to("cuda")
+            kw = dict(T=w.T, chunk_tokens=128, topk_idx=w.topk_idx, topk_logit=w.topk_logit,
+                      teacher_lse=w.teacher_lse, fuse_dlogits=case == "topk_fused_ds")
         outs = [ops.kl_fwd_bwd(w.H, w.W, **kw) for _ in range(2)]
         torch.cuda.synchronize()
         a, b = outs
@@ -40,14 +46,19 @@ def _worker(q):
         q.put(dict(error=repr(e)))
 
 
-def test_first_call_equals_second_in_fresh_processes():
+@pytest.mark.parametrize("case,processes", [("topk", PROCESSES), ("hidden", 2),
+                                            ("topk_fused_ds", 2)])
+def test_first_call_equals_second_in_fresh_processes(case, processes):
+    """topk: the case that exposed the staging race; hidden: the teacher-hidden
+    pass (both logit launches, fp32 teacher tile); topk_fused_ds: dS formed
+    inside the dH contraction and stored for dW."""
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     results = []
-    for _ in range(PROCESSES):
+    for _ in range(processes):
         q = ctx.Queue()
-        p = ctx.Process(target=_worker, args=(q,))
+        p = ctx.Process(target=_worker, args=(case, q))
         p.start()
         results.append(q.get(timeout=300))
         p.join(timeout=120)
