@@ -171,3 +171,54 @@ def test_random_vocabulary_shards_match_oracle(seed):
         r = ref[name]
         err = np.max(np.abs(out[name].double().cpu().numpy() - r))
         assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
+
+
+WIDE_CASES = 8
+
+
+@pytest.mark.parametrize("seed", range(WIDE_CASES))
+def test_random_wide_problem_matches_oracle(seed):
+    """Wide heads (d from 1024 to 4096, many short dW units per CTA pair, V
+    rarely a multiple of 256) with the options of _draw; fewer tokens so that
+    the oracle stays quick."""
+    rng = np.random.default_rng(9000 + seed)
+    w, o = _draw(100 + seed)
+    masked = w.mask is not None
+    d = 8 * int(rng.integers(128, 513))
+    N = min(w.N, 300)
+    V = min(w.V, 3000)
+    base = dict(T=w.T if not torch.is_tensor(w.T) else w.T[:N].cpu(), dtype=w.dtype,
+                w_std=0.02, seed=9500 + seed)
+    if w.mode == "topk":
+        w = wl.make_topk(f"rwide{seed}", N=N, d=d, V=V, K=min(w.K, V), d_t=w.d_t,
+                         tw_std=0.05, partial_mass=w.teacher_lse is not None, **base)
+    else:
+        w = wl.make_hidden(f"rwideh{seed}", N=N, d=d, d_t=w.d_t, V=V, tw_std=0.05, **base)
+    if masked:
+        w.mask = torch.from_numpy((rng.random(N) > 0.25).astype(np.uint8))
+    w = w.to("cuda")
+    kw = _kw(w, o)
+    if o["entry"] == "fused":
+        out = ops.kl_fwd_bwd(w.H, w.W, grad_loss=o["g"], fuse_dlogits=o["fuse"], **kw)
+        loss, dH, dW, wss = out["loss"], out["dH"], out["dW"], [out["workspace"]]
+    else:
+        keep = o["entry"] == "split_keep"
+        f = ops.kl_fwd(w.H, w.W, keep_last_chunk=keep, **kw)
+        b = ops.kl_bwd(w.H, w.W, f["lse_s"], f["lse_t"],
+                       grad_loss=torch.full((), o["g"], device="cuda"),
+                       workspace=f["workspace"] if keep else None, keep_last_chunk=keep, **kw)
+        loss, dH, dW, wss = f["loss"], b["dH"], b["dW"], [f["workspace"], b["workspace"]]
+    assert all(ops.status(ws) == 0 for ws in wss)
+    args = dict(T=w.T, mask=w.mask, mode=w.mode, grad_loss=o["g"], reverse_weight=o["beta"])
+    if w.mode == "topk":
+        args.update(topk_idx=w.topk_idx, topk_logit=w.topk_logit, teacher_lse=w.teacher_lse)
+    else:
+        args.update(Ht=w.Ht, Wt=w.Wt)
+    ref = oracle.kl_loss(w.H, w.W, **args)
+    case = f"wide seed {seed}: N={w.N} d={w.d} V={w.V} {w.mode} {w.dtype} {o}"
+    assert abs(loss.item() - ref["loss"]) <= 1e-3 * abs(ref["loss"]) + 1e-6, \
+        (case, loss.item(), ref["loss"])
+    for name, got in (("dH", dH), ("dW", dW)):
+        r = ref[name]
+        err = np.max(np.abs(got.double().cpu().numpy() - r))
+        assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
