@@ -371,11 +371,12 @@ Plan make_plan(const kl_problem* p, int entry) {
 }
 
 // ------------------------------------------------------------------ launches
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0>
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR = 0, int WIDE = 0, int XF = 0,
+          int EG = 1>
 int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& ma,
                 const CUtensorMap& mb, const CUtensorMap& mc, GemmParams gp, double flops,
                 const CUtensorMap* md = nullptr) {
-  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF>;
+  auto kern = gemm_tc_kernel<Elem, A_MN, B_MN, EPI, PAIR, WIDE, XF, EG>;
   static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -391,7 +392,7 @@ int launch_gemm(const char* name, cudaStream_t st, int sms, const CUtensorMap& m
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(XF ? kGemmThreadsXf : kGemmThreads);
+  cfg.blockDim = dim3((XF || EG == 2) ? kGemmThreadsXf : kGemmThreads);
   cfg.dynamicSmemBytes = kGemmSmemBytes;
   cfg.stream = st;
   if (PAIR) {
@@ -500,6 +501,14 @@ int gemm_logits(Ctx& c, const void* X, int64_t dx, const void* Wh, int64_t c0, i
   gp.tpart = tpart;
   gp.status = &c.sc->status;
   gp.spin_limit = spin_limit();
+  if constexpr (sizeof(Elem) == 2) {
+    // The student pass of the teacher-hidden mode reads the fp32 teacher tile
+    // and forms two exponentials per element: its epilogue outlasts a unit's
+    // MMAs, so two epilogue groups take alternate units.
+    if (tbuf != nullptr)
+      return launch_gemm<Elem, 0, 0, EPI_STATS, 1, 0, 0, 2>(name, c.st, c.sms, ma, mb, mc, gp,
+                                                            2.0 * Cn * p->V * dx);
+  }
   return launch_gemm<Elem, 0, 0, EPI_STATS, 1>(name, c.st, c.sms, ma, mb, mc, gp,
                                                2.0 * Cn * p->V * dx);
 }

@@ -48,6 +48,8 @@
 //              contraction then reads.  This is the dlogits step of the loss
 //              without its own pass over HBM (measured slower than that pass
 //              on B200 at d >= 2048, so it is opt-in).
+//   warps 6-9  (EG = 2 only, the teacher-hidden student pass) a second group
+//              of epilogue warps, taking every other unit.
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
 // the 512 columns with one 256 x 512 tile (see the template below).  In the
@@ -265,8 +267,14 @@ __device__ __forceinline__ void xf_row(uint8_t* rowp, int sw, __nv_bfloat162 sca
 // warps of both CTAs wait for them), the MMA issuer waits for the transforms
 // of both CTAs on a third ring of barriers, and a stage is refilled only after
 // the MMAs and the transform warps' dS stores (tmD) have read it.
-template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0>
-__global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
+// EG = 2 (bf16 statistics epilogues with a heavy per-element tail, the
+// student pass of the teacher-hidden mode): a second group of four epilogue
+// warps (6-9).  Group g takes every other unit of the CTA -- always the one
+// whose accumulator is TMEM buffer g -- so each unit's epilogue may last two
+// units' worth of MMAs.  The staging boxes are bf16 (2 KB).
+template <typename Elem, int A_MN, int B_MN, int EPI, int PAIR, int WIDE = 0, int XF = 0,
+          int EG = 1>
+__global__ void __launch_bounds__((XF || EG == 2) ? kGemmThreadsXf : kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC,
@@ -276,6 +284,9 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
   static_assert(!XF || (PAIR && sizeof(Elem) == 2 && A_MN == 0 &&
                         (EPI == EPI_STORE || EPI == EPI_ACCUM)),
                 "operand transform: bf16 2-CTA pairs, K-major A, store or accumulate");
+  static_assert(EG == 1 || (EG == 2 && EPI == EPI_STATS && PAIR && !WIDE && !XF &&
+                            sizeof(Elem) == 2),
+                "two epilogue groups: bf16 statistics epilogues on 2-CTA pairs");
   constexpr int kCtas = PAIR ? 2 : 1;
   constexpr int kHalves = WIDE ? 2 : 1;               // N = 256 MMAs per K step
   constexpr int kTileN = kBN * kHalves;               // output columns per unit
@@ -551,13 +562,18 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       bulk_wait_all();  // the dS stores have landed before exit
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 4 || (EG == 2 && warp >= 6)) {
     // ------------------------------------------------------------ epilogue
     // Each warp stages its 32 rows x 32 columns of output in shared memory
     // (two buffers, swizzled to match the output map) and one lane issues a TMA
     // bulk store -- an fp32 add-reduction into global memory when accumulating.
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    uint8_t* stg = staging + warp * 2 * kStageOutBytes;
+    // A warp reads the TMEM lanes of its quadrant (warp mod 4); with EG = 2,
+    // warps 6-9 form group 1 and cover the quadrants 2, 3, 0, 1.
+    const int quad = warp & 3;
+    const int group = warp < 4 ? 0 : 1;
+    constexpr int kBoxStride = EG == 2 ? kStageOutBytes / 2 : kStageOutBytes;  // bf16 only
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    uint8_t* stg = staging + (warp < 4 ? warp : warp - 2) * 2 * kBoxStride;
     const uint64_t out_policy = l2_policy_evict_first();
     uint32_t nbox = 0;  // output boxes this warp has staged
     uint32_t local = 0;
@@ -583,7 +599,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     auto store_box = [&](const uint32_t(&v)[32], float scale, float shift, int x, int y,
                          bool fp32_out, bool reduce, bool issue) {
       if (!issue) return;
-      uint8_t* sb = stg + (nbox & 1u) * kStageOutBytes;
+      uint8_t* sb = stg + (nbox & 1u) * kBoxStride;
       ++nbox;
       if (lane == 0) bulk_wait_read_1();  // the store that last used sb has read it
       __syncwarp();
@@ -619,6 +635,8 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
     };
     constexpr bool kElemF32 = sizeof(Elem) == 4;
     for (int t = unit; t < total_tiles; t += units, ++local) {
+      // EG = 2: group g takes the units whose accumulator is buffer g
+      if (EG == 2 && static_cast<int>(local & 1u) != group) continue;
       const UnitRange ur = unit_range(t, p);
       int tm, tn;
       tile_coords(ur.tile, p, tm, tn);
@@ -628,7 +646,7 @@ __global__ void __launch_bounds__(XF ? kGemmThreadsXf : kGemmThreads, 1)
       __syncwarp();
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_base + buf * kBN;
-      const int row0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM + warp * 32;
+      const int row0 = tm * kBM * kCtas + static_cast<int>(rank) * kBM + quad * 32;
       const int grow = row0 + lane;
       const bool rv = grow < p.rows_valid;
       const bool warp_rows = row0 < p.rows_valid;  // any row of this warp's box exists
