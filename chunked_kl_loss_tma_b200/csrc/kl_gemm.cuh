@@ -35,8 +35,9 @@
 // epilogue reads its own 128 accumulator rows from its own TMEM.  The pair
 // halves the operand bytes each SM stages per MMA.
 //
-// Roles (192 threads, one CTA per SM, grid-strided over output tiles):
-//   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 w + t
+// Roles (192 threads, 320 with XF or EG = 2; one CTA per SM, grid-strided over
+// output tiles):
+//   warps 0-3  epilogue: thread t of warp w owns accumulator row 32 (w mod 4) + t
 //              (TMEM lane), reads 32 fp32 columns per tcgen05.ld;
 //   warp 4     TMA producer (one thread): STAGES-deep ring of A/B tiles;
 //   warp 5     TMEM allocator + MMA issuer (one thread);
@@ -52,8 +53,8 @@
 //              of epilogue warps, taking every other unit.
 // Two 256-column accumulators in TMEM (512 columns) let the epilogue of tile
 // i overlap the main loop of tile i + 1; the WIDE variant (dH) instead fills
-// the 512 columns with one 256 x 512 tile (see the template below).  In the
-// waiting threads are parked by the hardware between barrier polls rather than
+// the 512 columns with one 256 x 512 tile (see the template below).  Waiting
+// threads are parked by the hardware between barrier polls rather than
 // spinning.
 //
 // Every wait on an mbarrier is bounded (spin_limit clock cycles); when one
