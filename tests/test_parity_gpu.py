@@ -454,6 +454,26 @@ def test_wide_heads(mode, d, d_t):
 
 
 @pytest.mark.parametrize("mode", ["topk", "hidden"])
+def test_vocabulary_262144(mode):
+    """A 2^18-entry vocabulary (1024 tiles of 256 columns per row, twice the
+    bench's): the split-V merge over all tiles, cache ids up to 262143 and the
+    gradients, fused call with a ragged chunk."""
+    V = 262144
+    if mode == "topk":
+        w = wl.make_topk("v256k", N=200, d=128, V=V, K=64, d_t=64, T=1.2, dtype=torch.bfloat16,
+                         w_std=0.1, tw_std=0.2, seed=43).to("cuda")
+    else:
+        w = wl.make_hidden("v256kh", N=200, d=128, d_t=96, V=V, T=1.7, dtype=torch.bfloat16,
+                           w_std=0.1, tw_std=0.1, seed=44).to("cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, want_row_loss=True, **_kw(w, chunk=128))
+    assert ops.status(out["workspace"]) == 0
+    ref = _oracle(w)
+    _check_loss(out["loss"].item(), ref["loss"])
+    _check_grad(out["dH"], ref["dH"], "dH")
+    _check_grad(out["dW"], ref["dW"], "dW")
+
+
+@pytest.mark.parametrize("mode", ["topk", "hidden"])
 def test_vocabulary_smaller_than_one_tile(mode):
     if mode == "topk":
         w = wl.make_topk("v40", N=70, d=32, V=40, K=40, d_t=16, T=0.9, dtype=torch.bfloat16,
