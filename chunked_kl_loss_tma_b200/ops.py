@@ -23,7 +23,9 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _need(t, name, dtype=None, device=None):
+def _need(t, name, dtype=None, device=None, shape=None):
+    """Check a tensor argument (None passes).  The C ABI takes bare pointers and
+    cannot see sizes, so every shape the kernels rely on is checked here."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
@@ -32,9 +34,18 @@ def _need(t, name, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t
+
+
+def _workspace(ws, device):
+    """A caller's workspace: a contiguous device tensor; its size in bytes (the
+    library checks it against kl_workspace_bytes)."""
+    _need(ws, "workspace", device=device)
+    return ws.numel() * ws.element_size()
 
 
 def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teacher_lse=None,
@@ -60,7 +71,7 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
         raise ValueError("H must be [N, d] and W [V, d]")
     if mask is not None and mask.dtype == torch.bool:
         mask = mask.view(torch.uint8)
-    _need(mask, "mask", torch.uint8, dev)
+    _need(mask, "mask", torch.uint8, dev, shape=(H.shape[0],))
     p = L.KLProblem()
     p.N, p.d = H.shape
     p.V = W.shape[0]
@@ -96,7 +107,7 @@ def make_problem(H, W, *, T=1.0, mask=None, topk_idx=None, topk_logit=None, teac
             raise ValueError("give either topk_idx/topk_logit or Ht/Wt")
         _need(topk_idx, "topk_idx", torch.int32, dev)
         _need(topk_logit, "topk_logit", torch.float32, dev)
-        _need(teacher_lse, "teacher_lse", torch.float32, dev)
+        _need(teacher_lse, "teacher_lse", torch.float32, dev, shape=(H.shape[0],))
         if topk_idx.shape != topk_logit.shape or topk_idx.shape[0] != H.shape[0]:
             raise ValueError("topk_idx and topk_logit must both be [N, K]")
         p.teacher = L.KL_TEACHER_TOPK
@@ -134,8 +145,8 @@ def kl_fwd_bwd(H, W, *, grad_loss=1.0, dW=None, accumulate_dW=False, want_row_lo
     if dW is None:
         dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
         accumulate_dW = False
-    _need(dW, "dW", torch.float32, dev)
-    L.check(L.kl_fwd_bwd(p, ws.data_ptr(), ws.numel(), grad_loss, loss.data_ptr(),
+    _need(dW, "dW", torch.float32, dev, shape=W.shape)
+    L.check(L.kl_fwd_bwd(p, ws.data_ptr(), _workspace(ws, dev), grad_loss, loss.data_ptr(),
                          _ptr(row_loss), dH.data_ptr(), dW.data_ptr(), accumulate_dW,
                          _stream(dev)), "kl_fwd_bwd")
     return dict(loss=loss, row_loss=row_loss, dH=dH, dW=dW, workspace=ws)
@@ -151,7 +162,7 @@ def kl_fwd(H, W, *, workspace=None, want_row_loss=True, **kw):
     lse_s = torch.empty(N, dtype=torch.float32, device=dev)
     lse_t = torch.empty(N, dtype=torch.float32, device=dev) if kw.get("Ht") is not None else None
     row_loss = torch.empty(N, dtype=torch.float32, device=dev) if want_row_loss else None
-    L.check(L.kl_fwd(p, ws.data_ptr(), ws.numel(), loss.data_ptr(), lse_s.data_ptr(),
+    L.check(L.kl_fwd(p, ws.data_ptr(), _workspace(ws, dev), loss.data_ptr(), lse_s.data_ptr(),
                      _ptr(lse_t), _ptr(row_loss), _stream(dev)), "kl_fwd")
     return dict(loss=loss, lse_s=lse_s, lse_t=lse_t, row_loss=row_loss, workspace=ws)
 
@@ -167,12 +178,19 @@ def kl_bwd(H, W, lse_s, lse_t=None, *, grad_loss=None, dW=None, accumulate_dW=Fa
     ws = workspace if workspace is not None else alloc_workspace(p, L.KL_ENTRY_BWD, dev)
     if grad_loss is None:
         grad_loss = torch.ones((), dtype=torch.float32, device=dev)
-    grad_loss = _need(grad_loss.to(torch.float32).contiguous(), "grad_loss", torch.float32, dev)
+    grad_loss = _need(grad_loss.to(torch.float32).reshape(()).contiguous(), "grad_loss",
+                      torch.float32, dev)
+    N = H.shape[0]
+    _need(lse_s, "lse_s", torch.float32, dev, shape=(N,))
+    if p.teacher == L.KL_TEACHER_HIDDEN and lse_t is None:
+        raise ValueError("lse_t (from kl_fwd) is required in the teacher-hidden mode")
+    _need(lse_t, "lse_t", torch.float32, dev, shape=(N,))
     dH = torch.empty_like(H)
     if dW is None:
         dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
         accumulate_dW = False
-    L.check(L.kl_bwd(p, ws.data_ptr(), ws.numel(), lse_s.data_ptr(), _ptr(lse_t),
+    _need(dW, "dW", torch.float32, dev, shape=W.shape)
+    L.check(L.kl_bwd(p, ws.data_ptr(), _workspace(ws, dev), lse_s.data_ptr(), _ptr(lse_t),
                      grad_loss.data_ptr(), dH.data_ptr(), dW.data_ptr(), accumulate_dW,
                      _stream(dev)), "kl_bwd")
     return dict(dH=dH, dW=dW, workspace=ws)

@@ -106,7 +106,7 @@ class ShardPass:
         """Chunk k's logits over the shard; returns its row statistics [rows, 2]."""
         rows = self.chunks[k][1]
         st = self._stats[:rows]
-        L.check(L.kl_vp_fwd_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel(), st.data_ptr(),
+        L.check(L.kl_vp_fwd_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel() * self.ws.element_size(), st.data_ptr(),
                                   self._stream), "kl_vp_fwd_chunk")
         return st
 
@@ -116,7 +116,7 @@ class ShardPass:
         if stats_all.shape != (P * rows, 2) or not stats_all.is_contiguous():
             raise ValueError("stats_all must be a contiguous [P * rows, 2] tensor")
         out = self._sums[:rows]
-        L.check(L.kl_vp_mid_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel(),
+        L.check(L.kl_vp_mid_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel() * self.ws.element_size(),
                                   stats_all.data_ptr(), P, rank, out.data_ptr(), self._stream),
                 "kl_vp_mid_chunk")
         return out
@@ -128,7 +128,7 @@ class ShardPass:
         for t in (stats_all,) + ((sums_all,) if self.two_exchanges else ()):
             if t is None or t.shape != (P * rows, 2) or not t.is_contiguous():
                 raise ValueError("statistics must be contiguous [P * rows, 2] tensors")
-        L.check(L.kl_vp_bwd_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel(),
+        L.check(L.kl_vp_bwd_chunk(self.p, k, self.ws.data_ptr(), self.ws.numel() * self.ws.element_size(),
                                   stats_all.data_ptr(), ops._ptr(sums_all), P, rank, grad_loss,
                                   self.loss.data_ptr(), ops._ptr(self.lse_s),
                                   ops._ptr(self.row_loss), self.dH32.data_ptr(),

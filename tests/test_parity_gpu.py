@@ -334,6 +334,39 @@ def test_launch_counter_and_profile():
     assert prof["gemm_teacher_logits"]["launches"] == prof["gemm_logits_stats"]["launches"] == chunks
 
 
+def test_binding_rejects_wrong_shapes():
+    """The C ABI sees bare pointers, so the binding checks every size the
+    kernels rely on and raises before anything is launched."""
+    w = _small_topk(seed=28)
+    kw = _kw(w)
+    N, V = w.N, w.V
+    bad = [
+        dict(kw, mask=torch.ones(N - 1, dtype=torch.uint8, device="cuda")),
+        dict(kw, teacher_lse=torch.zeros(N + 1, device="cuda")),
+    ]
+    for k in bad:
+        with pytest.raises(ValueError):
+            ops.kl_fwd_bwd(w.H, w.W, **k)
+    with pytest.raises(ValueError):
+        ops.kl_fwd_bwd(w.H, w.W, dW=torch.zeros(V - 1, w.d, device="cuda"), **kw)
+    f = ops.kl_fwd(w.H, w.W, **kw)
+    with pytest.raises(ValueError):
+        ops.kl_bwd(w.H, w.W, f["lse_s"][:-1], **kw)
+    with pytest.raises(ValueError):
+        ops.kl_bwd(w.H, w.W, f["lse_s"], dW=torch.zeros(w.d, V, device="cuda"), **kw)
+    h = _small_hidden(seed=29)
+    fh = ops.kl_fwd(h.H, h.W, **_kw(h))
+    with pytest.raises(ValueError):
+        ops.kl_bwd(h.H, h.W, fh["lse_s"], None, **_kw(h))  # lse_t missing
+    # a workspace of another element type is measured in bytes
+    ws = torch.empty((ops.workspace_bytes(ops.make_problem(w.H, w.W, **kw)[0], 2) + 3) // 4,
+                     dtype=torch.float32, device="cuda")
+    out = ops.kl_fwd_bwd(w.H, w.W, workspace=ws, **kw)
+    assert ops.status(ws) == 0
+    ref = ops.kl_fwd_bwd(w.H, w.W, **kw)
+    assert torch.equal(out["dW"], ref["dW"])
+
+
 def test_bitwise_deterministic_across_calls():
     """Every reduction has a fixed order (per-row statistics, split-V merge,
     split-K parts, per-chunk dW add-reductions issued in chunk order), so two
