@@ -367,6 +367,32 @@ def test_binding_rejects_wrong_shapes():
     assert torch.equal(out["dW"], ref["dW"])
 
 
+def test_two_streams_concurrently():
+    """Two problems (one per teacher mode) enqueued at once on two streams, each
+    with its own workspace: the library keeps no device state outside the
+    workspace, so each result equals the same call run alone, bit for bit."""
+    a = _small_topk(seed=30)
+    b = _small_hidden(seed=31)
+    ka, kb = _kw(a, chunk=128), _kw(b, chunk=96)
+    ref_a = ops.kl_fwd_bwd(a.H, a.W, **ka)
+    ref_b = ops.kl_fwd_bwd(b.H, b.W, **kb)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            oa = ops.kl_fwd_bwd(a.H, a.W, **ka)
+        with torch.cuda.stream(s2):
+            ob = ops.kl_fwd_bwd(b.H, b.W, **kb)
+        outs.append((oa, ob))
+    torch.cuda.synchronize()
+    for oa, ob in outs:
+        assert ops.status(oa["workspace"]) == 0 and ops.status(ob["workspace"]) == 0
+        for k in ("loss", "dH", "dW"):
+            assert torch.equal(oa[k], ref_a[k]), ("topk", k)
+            assert torch.equal(ob[k], ref_b[k]), ("hidden", k)
+
+
 def test_bitwise_deterministic_across_calls():
     """Every reduction has a fixed order (per-row statistics, split-V merge,
     split-K parts, per-chunk dW add-reductions issued in chunk order), so two
