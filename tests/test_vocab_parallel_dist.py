@@ -162,14 +162,16 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_vocabulary_parallel_pass_matches_whole_head_oracle():
+@pytest.mark.parametrize("world", [2, 3])
+def test_vocabulary_parallel_pass_matches_whole_head_oracle(world):
+    """world ranks of gloo, each with its vocabulary shard (3 ranks: uneven shards)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=120) for _ in range(2)]
+    res = [q.get(timeout=120) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -278,14 +280,15 @@ def _hidden_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_reverse_kl_pass_with_two_exchanges_matches_oracle():
+@pytest.mark.parametrize("world", [2, 3])
+def test_reverse_kl_pass_with_two_exchanges_matches_oracle(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_hidden_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_hidden_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=120) for _ in range(2)]
+    res = [q.get(timeout=120) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
