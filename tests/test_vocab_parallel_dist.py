@@ -1,5 +1,5 @@
 """Host logic of the vocabulary-parallel pass on CPU: shard boundaries, and
-`run_pass` driving two gloo ranks (top-K mode with one exchange per chunk, and
+`run_pass` driving two and three gloo ranks (top-K mode with one exchange per chunk, and
 teacher-hidden mode with a reverse-KL weight and two exchanges).
 
 Each rank's per-chunk compute here is a small numpy stand-in written from the
