@@ -1,4 +1,4 @@
-"""World-size-2 gloo tests (CPU) of the multi-rank host logic: token shards,
+"""Gloo tests (CPU, world sizes 1 to 3) of the multi-rank host logic: token shards,
 the global normaliser and max-over-ranks timing.  Per-rank compute is the
 oracle here (no GPU); the claim tested is that shard results combined with the
 global count equal the single-process result."""
@@ -67,11 +67,13 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_shards_with_global_normalizer_match_single_process():
+@pytest.mark.parametrize("world", [2, 3])
+def test_rank_shards_with_global_normalizer_match_single_process(world):
+    """world ranks (3: shards of 5, 4 and 4 of the 13 tokens)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = q.get(timeout=120)
@@ -82,7 +84,7 @@ def test_two_rank_shards_with_global_normalizer_match_single_process():
     assert n_all == n_ref
     assert loss == pytest.approx(ref, rel=1e-12)
     assert dw_err < 1e-12
-    assert slowest == 2.0
+    assert slowest == float(world)
 
 
 def _reduce_worker(rank, world, port, q):
