@@ -1,4 +1,4 @@
-"""Token data-parallel form with the CUDA path: two processes share one GPU and
+"""Token data-parallel form with the CUDA path: two or three processes share one GPU and
 exchange over gloo (host-side collectives, so neither rank's kernels wait on
 the other's).  Each rank runs its token shard through kl_fwd_bwd with the
 global count of valid tokens as the normaliser; the head gradient and the loss
@@ -65,17 +65,20 @@ def _worker(rank, world, port, reduce, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("reduce", ["all_reduce", "reduce_scatter"])
-def test_two_token_shards_over_gloo_on_one_gpu(reduce):
+@pytest.mark.parametrize("reduce,world", [("all_reduce", 2), ("reduce_scatter", 2),
+                                          ("reduce_scatter", 3)])
+def test_token_shards_over_gloo_on_one_gpu(reduce, world):
+    """world processes (3: uneven token shards, and dW row blocks of a V that 3
+    does not divide)."""
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, reduce, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, reduce, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=300) for _ in range(2)]
+    res = [q.get(timeout=300) for _ in range(world)]
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
