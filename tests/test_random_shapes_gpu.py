@@ -16,6 +16,8 @@ whole problem.
 Tolerances as in the other parity tests: loss relative error <= 1e-3 (plus 1e-6
 absolute, for losses that are 0), gradients max-abs error <= 2e-2 * max|oracle
 gradient|."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -26,7 +28,9 @@ from chunked_kl_loss_tma_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
-CASES = 48
+# Seeds per family; a larger sweep: KL_RANDOM_CASES=1248 KL_RANDOM_WIDE_CASES=60
+# KL_RANDOM_VP_CASES=80 python -m pytest tests/test_random_shapes_gpu.py
+CASES = int(os.environ.get("KL_RANDOM_CASES", 48))
 
 
 def _draw(seed):
@@ -107,7 +111,7 @@ def test_random_problem_matches_oracle(seed):
         assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
 
 
-VP_CASES = 16
+VP_CASES = int(os.environ.get("KL_RANDOM_VP_CASES", 16))
 
 
 def _draw_vp(seed):
@@ -173,7 +177,7 @@ def test_random_vocabulary_shards_match_oracle(seed):
         assert err <= 2e-2 * np.max(np.abs(r)) + 1e-6, (case, name, err, np.max(np.abs(r)))
 
 
-WIDE_CASES = 8
+WIDE_CASES = int(os.environ.get("KL_RANDOM_WIDE_CASES", 8))
 
 
 @pytest.mark.parametrize("seed", range(WIDE_CASES))
