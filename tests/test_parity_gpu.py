@@ -224,12 +224,18 @@ def test_fused_dlogits_edge_cases(case):
     _check_grad(out["dW"] - base if acc else out["dW"], ref["dW"], "dW")
 
 
-def test_autograd_function_matches_oracle():
-    w = _small_topk(N=160, V=2100, masked=False)
+@pytest.mark.parametrize("mode,keep,chunk", [("topk", True, 0), ("topk", False, 64),
+                                             ("topk", True, 64), ("hidden", True, 64),
+                                             ("hidden", False, 64)])
+def test_autograd_function_matches_oracle(mode, keep, chunk):
+    """fused_kl_loss through autograd: kl_fwd then kl_bwd, with the last chunk's
+    logits kept between them or every chunk recomputed."""
+    w = _small_topk(N=160, V=2100, masked=False) if mode == "topk" else \
+        _small_hidden(N=160, V=2100, seed=33)
     H = w.H.clone().requires_grad_(True)
     W = w.W.clone().requires_grad_(True)
-    kw = _kw(w)
-    loss = ops.fused_kl_loss(H, W, **kw)
+    kw = _kw(w, chunk=chunk)
+    loss = ops.fused_kl_loss(H, W, keep_last_chunk=keep, **kw)
     (2.0 * loss).backward()
     ref = _oracle(w, grad_loss=2.0)
     _check_loss(loss.item(), ref["loss"])
